@@ -1,0 +1,169 @@
+/*
+ * llama_block.h — C ABI of a B200 (sm_100a) LLaMA pre-norm decoder block.
+ *
+ * The block is the pre-norm decoder layer of the "LMDrive 大语言模型（LLM）核心推理单元"
+ * page (§2.5 LlamaDecoderLayer) and of chapter 02 of "LLM 核心机制交互讲义":
+ *
+ *   X'  = X  + o_proj( causal_softmax( RoPE(Q) RoPE(K)^T / sqrt(d_h) ) V ),
+ *              with Q, K, V projected from h = RMSNorm(X; g_attn)
+ *   X'' = X' + down_proj( SiLU(gate_proj(h2)) * up_proj(h2) ),  h2 = RMSNorm(X'; g_mlp)
+ *
+ * with grouped-query attention (query head h reads KV head h / (n_heads/n_kv_heads),
+ * the repeat_kv grouping of §2.3) and a KV cache for decode (chapter 04 of the
+ * mechanics page: the cache holds keys after RoPE; a decode step at cache length L
+ * rotates its query and key at position L and appends k, v at index L).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *    densely packed, in the handle's (or the call's) dtype: LB_F32 = float,
+ *    LB_BF16 = bfloat16 (storage) with fp32 accumulation. There is no host path.
+ *  - Weights use the nn.Linear layout [out_features, in_features].
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Work is
+ *    enqueued asynchronously; the call returns after the enqueue.
+ *  - Argument errors are detected on the host before anything is enqueued and
+ *    return LB_ERR_INVALID_ARG / LB_ERR_UNSUPPORTED / LB_ERR_CACHE_FULL; the
+ *    reason is available from llama_block_last_error() (thread-local string).
+ *  - Device-side waits are bounded: a wait that runs out latches an error word on
+ *    the device instead of hanging; llama_block_sync_status() reads it.
+ *  - Restrictions: head_dim in {64, 128}; n_heads % n_kv_heads == 0;
+ *    n_heads * head_dim and d are multiples of 64 for LB_BF16; y must not alias x.
+ *  - A handle is not thread-safe: do not call it concurrently from several threads.
+ */
+#ifndef LLAMA_BLOCK_H
+#define LLAMA_BLOCK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LB_OK = 0,
+    LB_ERR_INVALID_ARG = 1,  /* null pointer, non-positive or inconsistent size */
+    LB_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. head_dim 96) */
+    LB_ERR_CUDA = 3,         /* a CUDA runtime call failed (message in last_error) */
+    LB_ERR_OOM = 4,          /* device allocation failed */
+    LB_ERR_CACHE_FULL = 5,   /* a sequence would grow beyond t_max */
+    LB_ERR_TIMEOUT = 6,      /* a bounded device wait ran out (see sync_status) */
+    LB_ERR_NO_WEIGHTS = 7    /* prefill/decode before llama_block_set_weights */
+} lb_status;
+
+typedef enum { LB_F32 = 0, LB_BF16 = 1 } lb_dtype;
+
+typedef struct llama_block llama_block; /* opaque, library-owned */
+
+/* Create a block handle (LMDrive page §2.3–2.5: hidden_size d, num_attention_heads,
+ * num_key_value_heads, head_dim, intermediate_size f; RMSNorm eps §2.1; RoPE base
+ * §2.2). `max_pos` sizes the RoPE cos/sin table (positions 0 .. max_pos-1), which
+ * the library builds in fp64 on the host. Allocates library-owned device memory
+ * (packed weights, RoPE table, error word) on the current device.
+ * Returns LB_ERR_INVALID_ARG for non-positive sizes or a null `out`,
+ * LB_ERR_UNSUPPORTED for head_dim not in {64,128} or n_heads % n_kv_heads != 0. */
+lb_status llama_block_create(int d, int n_heads, int n_kv_heads, int head_dim, int f,
+                             float eps, float rope_base, lb_dtype dtype, int max_pos,
+                             llama_block** out);
+
+/* Copy and pack the block weights (device pointers, nn.Linear [out,in] layout,
+ * handle dtype): wq [H*dh, d], wk/wv [Hkv*dh, d], wo [d, H*dh], w_gate/w_up [f, d],
+ * w_down [d, f], g_attn/g_mlp [d] (input_layernorm / post_attention_layernorm
+ * weights). The library keeps its own packed copies (fused Q|K|V rows; gate/up
+ * rows interleaved in blocks of 128), so the caller may free its buffers once
+ * `stream` has passed this call. */
+lb_status llama_block_set_weights(llama_block* blk, const void* wq, const void* wk,
+                                  const void* wv, const void* wo, const void* w_gate,
+                                  const void* w_up, const void* w_down,
+                                  const void* g_attn, const void* g_mlp, void* stream);
+
+/* Preallocate the workspace for up to `max_tokens` prefill rows (B*T) and
+ * `max_batch` decode sequences, so that later calls allocate nothing (needed
+ * before capturing calls in a CUDA graph). Optional: calls grow the workspace
+ * on demand otherwise. */
+lb_status llama_block_reserve(llama_block* blk, int max_tokens, int max_batch);
+
+/* Prefill (LMDrive page §2.5 forward, positions 0..T-1 for every sequence).
+ * x, y: [B, T, d]. k_cache, v_cache: [B, n_kv_heads, t_max, head_dim] (caller-owned);
+ * K (after RoPE) and V of positions 0..T-1 are written to indices 0..T-1.
+ * cache_len: device int32 [B], set to T. T <= t_max and T <= max_pos required
+ * (else LB_ERR_CACHE_FULL). The host-side length mirror is set to T. */
+lb_status llama_block_prefill(llama_block* blk, const void* x, void* y, int B, int T,
+                              void* k_cache, void* v_cache, int t_max, int32_t* cache_len,
+                              void* stream);
+
+/* One decode step for B sequences with one new token each (mechanics page,
+ * chapter 04 KV-cache equation). x, y: [B, 1, d]. The new token of sequence b sits
+ * at position L_b = cache_len[b]; its rotated k and its v are written to cache
+ * index L_b, the query attends keys 0..L_b, and cache_len[b] becomes L_b + 1.
+ * The host mirror of the lengths (set by prefill or llama_block_set_lengths) is
+ * checked first: L_b + 1 > t_max or L_b >= max_pos returns LB_ERR_CACHE_FULL. */
+lb_status llama_block_decode(llama_block* blk, const void* x, void* y, int B,
+                             void* k_cache, void* v_cache, int t_max, int32_t* cache_len,
+                             void* stream);
+
+/* Tell the handle the current cache lengths (host array of B entries) when the
+ * caller filled the cache itself; the device cache_len array stays the caller's
+ * to set. */
+lb_status llama_block_set_lengths(llama_block* blk, const int32_t* lens_host, int B);
+
+/* KV-cache bytes of one block (mechanics page, chapter 04 memory accounting with
+ * L = 1): 2 * B * t_max * n_kv_heads * head_dim * sizeof(dtype). Host-only; 0 for
+ * invalid arguments. */
+size_t llama_block_kv_cache_bytes(int B, int n_kv_heads, int head_dim, int t_max,
+                                  lb_dtype dtype);
+
+/* Synchronise `stream`, read and clear the device error word (of the handle, or
+ * of the standalone entry points when blk is NULL). Returns LB_OK, LB_ERR_TIMEOUT
+ * (a bounded wait ran out, or a device-side bounds guard fired; details in
+ * last_error) or LB_ERR_CUDA. */
+lb_status llama_block_sync_status(llama_block* blk, void* stream);
+
+/* Free the handle and everything it owns (synchronises the device first). */
+void llama_block_destroy(llama_block* blk);
+
+/* Thread-local description of the last error (never NULL). */
+const char* llama_block_last_error(void);
+
+/* Self-test of the bounded-wait machinery: launch one kernel that waits on a
+ * device barrier that nothing completes, with a budget of `budget_ns`
+ * nanoseconds. The kernel gives up, latches the standalone error word and exits;
+ * llama_block_sync_status(NULL, stream) then returns LB_ERR_TIMEOUT. No GPU fault
+ * or hang is involved. */
+lb_status llama_block_selftest_timeout(long long budget_ns, void* stream);
+
+/* ---------------- standalone entry points (testing) ---------------- */
+
+/* RMSNorm (LMDrive page §2.1; mechanics page §02.3): y = g * x / sqrt(mean(x^2) + eps)
+ * over the last axis, fp32 accumulation, one rounding. x, y: [rows, d]; g: [d]. */
+lb_status rmsnorm(const void* x, const void* g, void* y, int rows, int d, float eps,
+                  lb_dtype dtype, void* stream);
+
+/* RoPE in place (LMDrive page §2.2, half-split rotate_half pairing):
+ * x: [B, n_heads, T, head_dim]; pos: device int32 [B, T] positions (>= 0).
+ * Angles pos * base^(-2i/head_dim) are formed in fp64 on the device. */
+lb_status rope_apply(void* x, const int32_t* pos, int B, int T, int n_heads, int head_dim,
+                     float base, lb_dtype dtype, void* stream);
+
+/* Causal softmax attention with GQA (LMDrive page §2.3; mechanics page §02.1).
+ * q: [B, n_heads, Tq, head_dim]; k, v: [B, n_kv_heads, k_stride_T, head_dim] of which
+ * the first Tk rows are used; query row i sits at position Tk - Tq + i and attends
+ * keys 0 .. Tk - Tq + i. o: [B, Tq, n_heads * head_dim] (the layout o_proj reads).
+ * Scores are scaled by 1/sqrt(head_dim). Requires 1 <= Tq <= Tk <= k_stride_T. */
+lb_status causal_attn(const void* q, const void* k, const void* v, void* o, int B, int Tq,
+                      int Tk, int n_heads, int n_kv_heads, int head_dim, int k_stride_T,
+                      lb_dtype dtype, void* stream);
+
+/* SwiGLU MLP without residual (LMDrive page §2.4; Llama-MLP page §4.2):
+ * y = down( SiLU(h gate^T) * (h up^T) ). h, y: [M, d]; w_gate, w_up: [f, d];
+ * w_down: [d, f]. Packs the gate/up weights into a temporary device buffer per
+ * call (allocates and frees it). */
+lb_status swiglu_mlp(const void* h, const void* w_gate, const void* w_up,
+                     const void* w_down, void* y, int M, int d, int f, lb_dtype dtype,
+                     void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLAMA_BLOCK_H */

@@ -1,0 +1,241 @@
+"""Python binding of the B200 LLaMA pre-norm decoder block library.
+
+A thin ctypes layer over ``libllama_block.so`` (the C ABI declared in
+``include/llama_block.h``): every function here has the C name, checks and
+marshals its arguments (torch tensors -> device pointers, the current CUDA
+stream -> ``cudaStream_t``) and raises :class:`LlamaBlockError` on a non-OK
+status. All computation runs in the library's CUDA kernels; there is no CPU
+path, and importing this package fails loudly when the library is not built.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from pathlib import Path
+
+import torch
+
+__all__ = [
+    "LB_F32", "LB_BF16", "LlamaBlockError", "lib", "lib_path", "dtype_code",
+    "llama_block_create", "llama_block_set_weights", "llama_block_reserve",
+    "llama_block_prefill", "llama_block_decode", "llama_block_set_lengths",
+    "llama_block_kv_cache_bytes", "llama_block_sync_status", "llama_block_destroy",
+    "llama_block_last_error", "llama_block_selftest_timeout",
+    "rmsnorm", "rope_apply", "causal_attn", "swiglu_mlp", "LlamaBlock",
+]
+
+LB_F32, LB_BF16 = 0, 1
+STATUS = {0: "LB_OK", 1: "LB_ERR_INVALID_ARG", 2: "LB_ERR_UNSUPPORTED", 3: "LB_ERR_CUDA",
+          4: "LB_ERR_OOM", 5: "LB_ERR_CACHE_FULL", 6: "LB_ERR_TIMEOUT", 7: "LB_ERR_NO_WEIGHTS"}
+
+lib_path = Path(os.environ.get("LLAMA_BLOCK_LIB", Path(__file__).resolve().parent / "libllama_block.so"))
+if not lib_path.exists():
+    raise ImportError(
+        f"llama_pre_norm_b200: CUDA library {lib_path} is not built "
+        "(run `python -m llama_pre_norm_b200.build`); there is no fallback path")
+lib = ctypes.CDLL(str(lib_path))
+
+_p, _i, _f, _sz, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_longlong
+_pp = ctypes.POINTER(ctypes.c_void_p)
+_SIGS = {
+    "llama_block_create": (_i, [_i, _i, _i, _i, _i, _f, _f, _i, _i, _pp]),
+    "llama_block_set_weights": (_i, [_p] * 11),
+    "llama_block_reserve": (_i, [_p, _i, _i]),
+    "llama_block_prefill": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p]),
+    "llama_block_decode": (_i, [_p, _p, _p, _i, _p, _p, _i, _p, _p]),
+    "llama_block_set_lengths": (_i, [_p, _p, _i]),
+    "llama_block_kv_cache_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "llama_block_sync_status": (_i, [_p, _p]),
+    "llama_block_destroy": (None, [_p]),
+    "llama_block_last_error": (ctypes.c_char_p, []),
+    "llama_block_selftest_timeout": (_i, [_ll, _p]),
+    "rmsnorm": (_i, [_p, _p, _p, _i, _i, _f, _i, _p]),
+    "rope_apply": (_i, [_p, _p, _i, _i, _i, _i, _f, _i, _p]),
+    "causal_attn": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p]),
+    "swiglu_mlp": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _p]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class LlamaBlockError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+        msg = lib.llama_block_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {self.name}: {msg}")
+
+
+def _check(st: int, where: str) -> None:
+    if st != 0:
+        raise LlamaBlockError(st, where)
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return LB_F32
+    if dt == torch.bfloat16:
+        return LB_BF16
+    raise TypeError(f"unsupported dtype {dt} (float32 or bfloat16)")
+
+
+def _ptr(t: torch.Tensor | None, name: str, dtype=None) -> int | None:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+# ----------------------------------------------------------------- handle API
+def llama_block_create(d, n_heads, n_kv_heads, head_dim, f, eps, rope_base, dtype, max_pos) -> int:
+    out = ctypes.c_void_p()
+    code = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    _check(lib.llama_block_create(d, n_heads, n_kv_heads, head_dim, f, eps, rope_base, code, max_pos,
+                                  ctypes.byref(out)), "llama_block_create")
+    return out.value
+
+
+def llama_block_set_weights(h, wq, wk, wv, wo, w_gate, w_up, w_down, g_attn, g_mlp, stream=None):
+    dt = wq.dtype
+    ptrs = [_ptr(t, n, dt) for t, n in ((wq, "wq"), (wk, "wk"), (wv, "wv"), (wo, "wo"),
+                                         (w_gate, "w_gate"), (w_up, "w_up"), (w_down, "w_down"),
+                                         (g_attn, "g_attn"), (g_mlp, "g_mlp"))]
+    _check(lib.llama_block_set_weights(h, *ptrs, _stream(stream)), "llama_block_set_weights")
+
+
+def llama_block_reserve(h, max_tokens, max_batch):
+    _check(lib.llama_block_reserve(h, max_tokens, max_batch), "llama_block_reserve")
+
+
+def llama_block_prefill(h, x, y, k_cache, v_cache, cache_len, stream=None):
+    B, T, _ = x.shape
+    t_max = k_cache.shape[2]
+    _check(lib.llama_block_prefill(h, _ptr(x, "x"), _ptr(y, "y", x.dtype), B, T,
+                                   _ptr(k_cache, "k_cache", x.dtype), _ptr(v_cache, "v_cache", x.dtype),
+                                   t_max, _ptr(cache_len, "cache_len", torch.int32), _stream(stream)),
+           "llama_block_prefill")
+
+
+def llama_block_decode(h, x, y, k_cache, v_cache, cache_len, stream=None):
+    B = x.shape[0]
+    t_max = k_cache.shape[2]
+    _check(lib.llama_block_decode(h, _ptr(x, "x"), _ptr(y, "y", x.dtype), B,
+                                  _ptr(k_cache, "k_cache", x.dtype), _ptr(v_cache, "v_cache", x.dtype),
+                                  t_max, _ptr(cache_len, "cache_len", torch.int32), _stream(stream)),
+           "llama_block_decode")
+
+
+def llama_block_set_lengths(h, lens):
+    arr = (ctypes.c_int32 * len(lens))(*[int(v) for v in lens])
+    _check(lib.llama_block_set_lengths(h, arr, len(lens)), "llama_block_set_lengths")
+
+
+def llama_block_kv_cache_bytes(B, n_kv_heads, head_dim, t_max, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    return int(lib.llama_block_kv_cache_bytes(B, n_kv_heads, head_dim, t_max, code))
+
+
+def llama_block_sync_status(h=None, stream=None):
+    _check(lib.llama_block_sync_status(h, _stream(stream)), "llama_block_sync_status")
+
+
+def llama_block_destroy(h):
+    lib.llama_block_destroy(h)
+
+
+def llama_block_last_error() -> str:
+    return lib.llama_block_last_error().decode(errors="replace")
+
+
+def llama_block_selftest_timeout(budget_ns: int, stream=None):
+    _check(lib.llama_block_selftest_timeout(int(budget_ns), _stream(stream)), "llama_block_selftest_timeout")
+
+
+# ----------------------------------------------------------------- standalone entry points
+def rmsnorm(x, g, y, eps, stream=None):
+    d = x.shape[-1]
+    rows = x.numel() // d
+    _check(lib.rmsnorm(_ptr(x, "x"), _ptr(g, "g", x.dtype), _ptr(y, "y", x.dtype), rows, d, eps,
+                       dtype_code(x.dtype), _stream(stream)), "rmsnorm")
+
+
+def rope_apply(x, pos, base, stream=None):
+    B, H, T, dh = x.shape
+    _check(lib.rope_apply(_ptr(x, "x"), _ptr(pos, "pos", torch.int32), B, T, H, dh, base,
+                          dtype_code(x.dtype), _stream(stream)), "rope_apply")
+
+
+def causal_attn(q, k, v, o, Tk=None, stream=None):
+    B, H, Tq, dh = q.shape
+    Hkv, k_stride = k.shape[1], k.shape[2]
+    Tk = k_stride if Tk is None else Tk
+    _check(lib.causal_attn(_ptr(q, "q"), _ptr(k, "k", q.dtype), _ptr(v, "v", q.dtype),
+                           _ptr(o, "o", q.dtype), B, Tq, Tk, H, Hkv, dh, k_stride,
+                           dtype_code(q.dtype), _stream(stream)), "causal_attn")
+
+
+def swiglu_mlp(h, w_gate, w_up, w_down, y, stream=None):
+    d = h.shape[-1]
+    M = h.numel() // d
+    f = w_gate.shape[0]
+    _check(lib.swiglu_mlp(_ptr(h, "h"), _ptr(w_gate, "w_gate", h.dtype), _ptr(w_up, "w_up", h.dtype),
+                          _ptr(w_down, "w_down", h.dtype), _ptr(y, "y", h.dtype), M, d, f,
+                          dtype_code(h.dtype), _stream(stream)), "swiglu_mlp")
+
+
+class LlamaBlock:
+    """Owns a ``llama_block`` handle (create / set_weights / prefill / decode)."""
+
+    def __init__(self, d, n_heads, n_kv_heads, head_dim, f, eps=1e-6, rope_base=10000.0,
+                 dtype=torch.bfloat16, max_pos=4096):
+        self.d, self.n_heads, self.n_kv_heads, self.head_dim, self.f = d, n_heads, n_kv_heads, head_dim, f
+        self.dtype = dtype
+        self.max_pos = max_pos
+        self.handle = llama_block_create(d, n_heads, n_kv_heads, head_dim, f, eps, rope_base,
+                                         dtype_code(dtype), max_pos)
+
+    def set_weights(self, w: dict, stream=None):
+        llama_block_set_weights(self.handle, w["wq"], w["wk"], w["wv"], w["wo"], w["w_gate"],
+                                w["w_up"], w["w_down"], w["g_attn"], w["g_mlp"], stream)
+
+    def reserve(self, max_tokens, max_batch):
+        llama_block_reserve(self.handle, max_tokens, max_batch)
+
+    def prefill(self, x, y, k_cache, v_cache, cache_len, stream=None):
+        llama_block_prefill(self.handle, x, y, k_cache, v_cache, cache_len, stream)
+
+    def decode(self, x, y, k_cache, v_cache, cache_len, stream=None):
+        llama_block_decode(self.handle, x, y, k_cache, v_cache, cache_len, stream)
+
+    def set_lengths(self, lens):
+        llama_block_set_lengths(self.handle, lens)
+
+    def sync_status(self, stream=None):
+        llama_block_sync_status(self.handle, stream)
+
+    def close(self):
+        if self.handle:
+            llama_block_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

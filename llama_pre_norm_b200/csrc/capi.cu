@@ -1,0 +1,685 @@
+// capi.cu — the C ABI of the library (include/llama_block.h): handle lifecycle,
+// weight packing, RoPE table, workspace, and the launch sequences of prefill and
+// decode. Host code only; every step of the block runs in the kernels of the
+// other translation units.
+//
+// Prefill of the pre-norm layer (LMDrive page §2.5), bf16:
+//   rmsnorm(X) -> h | tcgen05 GEMM h·Wqkv^T with RoPE + Q/K/V scatter | tcgen05 flash
+//   attention -> O | GEMM O·Wo^T + X -> X' | rmsnorm(X') -> h2 |
+//   GEMM h2·Wgu^T with SiLU(g)*u -> A | GEMM A·Wd^T + X' -> X''.
+// Decode (chapter 04 of the mechanics page), bf16, B tokens: the same stages with
+// swap-AB split-K tcgen05 GEMMs (weights stream as the 128-row operand, the B
+// tokens are the N side), fp32 partials reduced by the small fused kernels, and
+// split-KV attention over the cache.
+// fp32 handles run the same stages on the fp32 SIMT kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/llama_block.h"
+#include "internal.h"
+
+using namespace lb;
+
+// ------------------------------------------------------------------ errors
+static thread_local std::string g_last_error = "no error";
+
+static lb_status fail(lb_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+#define LB_CUDA(call)                                                                     \
+  do {                                                                                    \
+    cudaError_t e_ = (call);                                                              \
+    if (e_ != cudaSuccess)                                                                \
+      return fail(e_ == cudaErrorMemoryAllocation ? LB_ERR_OOM : LB_ERR_CUDA, "%s: %s (%s:%d)", \
+                  #call, cudaGetErrorString(e_), __FILE__, __LINE__);                     \
+  } while (0)
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+namespace lb {
+
+bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc || (reinterpret_cast<uintptr_t>(base) & 15) || (cols * 2) % 16) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_3d_bf16(CUtensorMap* m, const void* base, uint64_t planes, uint64_t rows,
+                       uint64_t cols, uint64_t plane_stride, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc || (reinterpret_cast<uintptr_t>(base) & 15) || (cols * 2) % 16 ||
+      (plane_stride * 2) % 16)
+    return false;
+  cuuint64_t dims[3] = {cols, rows, planes};
+  cuuint64_t strides[2] = {cols * 2, plane_stride * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace lb
+
+// ------------------------------------------------------------------ device info
+static int num_sms_of_current_device() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+// Error word of the standalone entry points, one per device.
+static std::mutex g_err_mu;
+static std::map<int, int*> g_err_words;
+
+static int* standalone_err_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  auto it = g_err_words.find(dev);
+  if (it != g_err_words.end()) return it->second;
+  int* p = nullptr;
+  if (cudaMalloc(&p, sizeof(int)) != cudaSuccess) return nullptr;
+  if (cudaMemset(p, 0, sizeof(int)) != cudaSuccess) return nullptr;
+  g_err_words[dev] = p;
+  return p;
+}
+
+// ------------------------------------------------------------------ handle
+struct llama_block {
+  int d, H, Hkv, dh, f, max_pos, dtype, device, num_sms;
+  float eps, base;
+  size_t esz;
+  int n_qkv;   // (H + 2 Hkv) * dh
+  int f_pad;   // bf16: f rounded up to 128 (gate/up interleave block)
+  int n_gu;    // rows of the packed gate/up weight
+  void *w_qkv = nullptr, *w_o = nullptr, *w_gu = nullptr, *w_d = nullptr;
+  void *g1 = nullptr, *g2 = nullptr;
+  float *cos_t = nullptr, *sin_t = nullptr;
+  int* err = nullptr;
+  bool has_weights = false;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  std::vector<int> lens;  // host mirror of the cache lengths
+};
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace carving: each region 256-byte aligned.
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base((char*)b) {}
+  void* take(size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off = align_up(off + bytes, 256);
+    return p;
+  }
+};
+
+struct PrefillWs {
+  void *h, *q, *o, *x1, *a;
+  float *qkv32, *gu32;
+};
+struct DecodeWs {
+  void *h, *q, *o, *x1, *a;
+  float* part;
+  float* attn_part;
+};
+
+static int decode_split(int tiles, int K) {
+  const int KB = (K + 63) / 64;
+  int s = (296 + tiles - 1) / tiles;
+  s = std::max(1, std::min(s, std::max(1, KB / 4)));
+  return s;
+}
+
+static PrefillWs carve_prefill(const llama_block* b, void* base, int M, size_t* total) {
+  Carver c(base);
+  PrefillWs w;
+  w.h = c.take((size_t)M * b->d * b->esz);
+  w.q = c.take((size_t)M * b->H * b->dh * b->esz);
+  w.o = c.take((size_t)M * b->H * b->dh * b->esz);
+  w.x1 = c.take((size_t)M * b->d * b->esz);
+  w.a = c.take((size_t)M * b->f_pad * b->esz);
+  if (b->dtype == kF32) {
+    w.qkv32 = (float*)c.take((size_t)M * b->n_qkv * 4);
+    w.gu32 = (float*)c.take((size_t)M * b->n_gu * 4);
+  } else {
+    w.qkv32 = w.gu32 = nullptr;
+  }
+  *total = c.off;
+  return w;
+}
+
+static DecodeWs carve_decode(const llama_block* b, void* base, int B, int t_max, size_t* total) {
+  Carver c(base);
+  DecodeWs w;
+  w.h = c.take((size_t)B * b->d * b->esz);
+  w.q = c.take((size_t)B * b->H * b->dh * b->esz);
+  w.o = c.take((size_t)B * b->H * b->dh * b->esz);
+  w.x1 = c.take((size_t)B * b->d * b->esz);
+  w.a = c.take((size_t)B * b->f_pad * b->esz);
+  size_t part = 0;
+  if (b->dtype == kBF16) {
+    const int s1 = decode_split((b->n_qkv + 127) / 128, b->d);
+    const int s2 = decode_split((b->d + 127) / 128, b->H * b->dh);
+    const int s3 = decode_split((b->n_gu + 127) / 128, b->d);
+    const int s4 = decode_split((b->d + 127) / 128, b->f);
+    part = std::max({(size_t)s1 * B * b->n_qkv, (size_t)s2 * B * b->d, (size_t)s3 * B * b->n_gu,
+                     (size_t)s4 * B * b->d});
+  } else {
+    part = std::max((size_t)B * b->n_qkv, (size_t)B * b->n_gu);
+  }
+  w.part = (float*)c.take(part * 4);
+  w.attn_part = (float*)c.take((size_t)B * b->H * decode_attn_chunks(t_max) * (b->dh + 2) * 4);
+  *total = c.off;
+  return w;
+}
+
+static lb_status ensure_ws(llama_block* b, size_t need) {
+  if (need <= b->ws_bytes) return LB_OK;
+  if (b->ws) {
+    LB_CUDA(cudaDeviceSynchronize());
+    LB_CUDA(cudaFree(b->ws));
+    b->ws = nullptr;
+    b->ws_bytes = 0;
+  }
+  LB_CUDA(cudaMalloc(&b->ws, need));
+  b->ws_bytes = need;
+  return LB_OK;
+}
+
+extern "C" {
+
+const char* llama_block_last_error(void) { return g_last_error.c_str(); }
+
+size_t llama_block_kv_cache_bytes(int B, int n_kv_heads, int head_dim, int t_max, lb_dtype dtype) {
+  if (B <= 0 || n_kv_heads <= 0 || head_dim <= 0 || t_max <= 0) return 0;
+  if (dtype != LB_F32 && dtype != LB_BF16) return 0;
+  const size_t es = dtype == LB_F32 ? 4 : 2;
+  return (size_t)2 * B * t_max * n_kv_heads * head_dim * es;
+}
+
+lb_status llama_block_create(int d, int n_heads, int n_kv_heads, int head_dim, int f, float eps,
+                             float rope_base, lb_dtype dtype, int max_pos, llama_block** out) {
+  if (!out) return fail(LB_ERR_INVALID_ARG, "create: out is NULL");
+  *out = nullptr;
+  if (d <= 0 || n_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0 || f <= 0 || max_pos <= 0)
+    return fail(LB_ERR_INVALID_ARG, "create: sizes must be positive");
+  if (!(eps > 0.f) || !(rope_base > 0.f))
+    return fail(LB_ERR_INVALID_ARG, "create: eps and rope_base must be positive");
+  if (dtype != LB_F32 && dtype != LB_BF16) return fail(LB_ERR_INVALID_ARG, "create: bad dtype");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(LB_ERR_UNSUPPORTED, "create: head_dim %d not in {64,128}", head_dim);
+  if (n_heads % n_kv_heads != 0)
+    return fail(LB_ERR_UNSUPPORTED, "create: n_heads %% n_kv_heads != 0");
+  if (n_heads / n_kv_heads > 8)
+    return fail(LB_ERR_UNSUPPORTED, "create: more than 8 query heads per KV head");
+  if (d % 8 != 0 || d > 8192)
+    return fail(LB_ERR_UNSUPPORTED, "create: d must be a multiple of 8 and <= 8192");
+  if (dtype == LB_BF16 && (d % 64 != 0 || f % 8 != 0 || (n_heads * head_dim) % 64 != 0))
+    return fail(LB_ERR_UNSUPPORTED, "create: bf16 needs d %% 64 == 0 and f %% 8 == 0");
+
+  llama_block* b = new llama_block();
+  b->d = d;
+  b->H = n_heads;
+  b->Hkv = n_kv_heads;
+  b->dh = head_dim;
+  b->f = f;
+  b->max_pos = max_pos;
+  b->dtype = dtype;
+  b->eps = eps;
+  b->base = rope_base;
+  b->esz = dtype == LB_F32 ? 4 : 2;
+  b->n_qkv = (n_heads + 2 * n_kv_heads) * head_dim;
+  b->f_pad = dtype == LB_BF16 ? (f + 127) / 128 * 128 : f;
+  b->n_gu = 2 * b->f_pad;
+
+  auto cleanup_fail = [&](lb_status st) {
+    llama_block_destroy(b);
+    return st;
+  };
+  if (cudaGetDevice(&b->device) != cudaSuccess) {
+    cudaGetLastError();
+    delete b;
+    return fail(LB_ERR_CUDA, "create: no CUDA device");
+  }
+  b->num_sms = num_sms_of_current_device();
+  const size_t es = b->esz;
+  if (cudaMalloc(&b->w_qkv, (size_t)b->n_qkv * d * es) != cudaSuccess ||
+      cudaMalloc(&b->w_o, (size_t)d * n_heads * head_dim * es) != cudaSuccess ||
+      cudaMalloc(&b->w_gu, (size_t)b->n_gu * d * es) != cudaSuccess ||
+      cudaMalloc(&b->w_d, (size_t)d * f * es) != cudaSuccess ||
+      cudaMalloc(&b->g1, (size_t)d * es) != cudaSuccess ||
+      cudaMalloc(&b->g2, (size_t)d * es) != cudaSuccess ||
+      cudaMalloc(&b->cos_t, (size_t)max_pos * (head_dim / 2) * 4) != cudaSuccess ||
+      cudaMalloc(&b->sin_t, (size_t)max_pos * (head_dim / 2) * 4) != cudaSuccess ||
+      cudaMalloc(&b->err, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    fail(LB_ERR_OOM, "create: device allocation failed");
+    return cleanup_fail(LB_ERR_OOM);
+  }
+  // RoPE table (LMDrive page §2.2): inv_freq_i = base^(-2i/dh), angle = pos * inv_freq_i,
+  // formed in fp64 on the host and stored as fp32 cos / sin [max_pos][dh/2].
+  const int half = head_dim / 2;
+  std::vector<float> ct((size_t)max_pos * half), st((size_t)max_pos * half);
+  for (int i = 0; i < half; ++i) {
+    const double inv = 1.0 / std::pow((double)rope_base, (2.0 * i) / (double)head_dim);
+    for (int p = 0; p < max_pos; ++p) {
+      const double a = (double)p * inv;
+      ct[(size_t)p * half + i] = (float)std::cos(a);
+      st[(size_t)p * half + i] = (float)std::sin(a);
+    }
+  }
+  if (cudaMemcpy(b->cos_t, ct.data(), ct.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(b->sin_t, st.data(), st.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemset(b->err, 0, sizeof(int)) != cudaSuccess ||
+      cudaMemset(b->w_gu, 0, (size_t)b->n_gu * d * es) != cudaSuccess) {
+    cudaGetLastError();
+    fail(LB_ERR_CUDA, "create: device initialisation failed");
+    return cleanup_fail(LB_ERR_CUDA);
+  }
+  *out = b;
+  return LB_OK;
+}
+
+void llama_block_destroy(llama_block* b) {
+  if (!b) return;
+  cudaDeviceSynchronize();
+  for (void* p : {b->w_qkv, b->w_o, b->w_gu, b->w_d, b->g1, b->g2, (void*)b->cos_t,
+                  (void*)b->sin_t, (void*)b->err, b->ws})
+    if (p) cudaFree(p);
+  delete b;
+}
+
+lb_status llama_block_set_weights(llama_block* b, const void* wq, const void* wk, const void* wv,
+                                  const void* wo, const void* w_gate, const void* w_up,
+                                  const void* w_down, const void* g_attn, const void* g_mlp,
+                                  void* stream) {
+  if (!b) return fail(LB_ERR_INVALID_ARG, "set_weights: NULL handle");
+  if (!wq || !wk || !wv || !wo || !w_gate || !w_up || !w_down || !g_attn || !g_mlp)
+    return fail(LB_ERR_INVALID_ARG, "set_weights: NULL weight pointer");
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t es = b->esz, d = b->d;
+  const size_t nq = (size_t)b->H * b->dh, nkv = (size_t)b->Hkv * b->dh;
+  char* qkv = (char*)b->w_qkv;
+  // fused Q | K | V rows
+  LB_CUDA(cudaMemcpyAsync(qkv, wq, nq * d * es, cudaMemcpyDeviceToDevice, s));
+  LB_CUDA(cudaMemcpyAsync(qkv + nq * d * es, wk, nkv * d * es, cudaMemcpyDeviceToDevice, s));
+  LB_CUDA(cudaMemcpyAsync(qkv + (nq + nkv) * d * es, wv, nkv * d * es, cudaMemcpyDeviceToDevice, s));
+  LB_CUDA(cudaMemcpyAsync(b->w_o, wo, d * nq * es, cudaMemcpyDeviceToDevice, s));
+  LB_CUDA(cudaMemcpyAsync(b->w_d, w_down, d * b->f * es, cudaMemcpyDeviceToDevice, s));
+  LB_CUDA(cudaMemcpyAsync(b->g1, g_attn, d * es, cudaMemcpyDeviceToDevice, s));
+  LB_CUDA(cudaMemcpyAsync(b->g2, g_mlp, d * es, cudaMemcpyDeviceToDevice, s));
+  char* gu = (char*)b->w_gu;
+  if (b->dtype == kF32) {
+    // [gate ; up]
+    LB_CUDA(cudaMemcpyAsync(gu, w_gate, (size_t)b->f * d * es, cudaMemcpyDeviceToDevice, s));
+    LB_CUDA(cudaMemcpyAsync(gu + (size_t)b->f * d * es, w_up, (size_t)b->f * d * es,
+                            cudaMemcpyDeviceToDevice, s));
+  } else {
+    // blocks of 128 rows: [gate rows 128j.. | up rows 128j..] for j = 0, 1, ...
+    const size_t blk = 128 * d * es;
+    const int full_blocks = b->f / 128;
+    if (full_blocks > 0) {
+      LB_CUDA(cudaMemcpy2DAsync(gu, 2 * blk, w_gate, blk, blk, full_blocks,
+                                cudaMemcpyDeviceToDevice, s));
+      LB_CUDA(cudaMemcpy2DAsync(gu + blk, 2 * blk, w_up, blk, blk, full_blocks,
+                                cudaMemcpyDeviceToDevice, s));
+    }
+    const int rem = b->f - full_blocks * 128;
+    if (rem > 0) {
+      const size_t src = (size_t)full_blocks * blk;
+      LB_CUDA(cudaMemcpyAsync(gu + 2 * src, (const char*)w_gate + src, rem * d * es,
+                              cudaMemcpyDeviceToDevice, s));
+      LB_CUDA(cudaMemcpyAsync(gu + 2 * src + blk, (const char*)w_up + src, rem * d * es,
+                              cudaMemcpyDeviceToDevice, s));
+    }
+  }
+  b->has_weights = true;
+  return LB_OK;
+}
+
+lb_status llama_block_reserve(llama_block* b, int max_tokens, int max_batch) {
+  if (!b) return fail(LB_ERR_INVALID_ARG, "reserve: NULL handle");
+  if (max_tokens < 0 || max_batch < 0) return fail(LB_ERR_INVALID_ARG, "reserve: negative size");
+  size_t a = 0, c = 0;
+  carve_prefill(b, nullptr, max_tokens, &a);
+  carve_decode(b, nullptr, max_batch, b->max_pos, &c);
+  return ensure_ws(b, std::max(a, c));
+}
+
+lb_status llama_block_set_lengths(llama_block* b, const int32_t* lens_host, int B) {
+  if (!b || !lens_host || B <= 0) return fail(LB_ERR_INVALID_ARG, "set_lengths: bad argument");
+  b->lens.assign(lens_host, lens_host + B);
+  return LB_OK;
+}
+
+static lb_status check_cache_args(llama_block* b, const void* x, const void* y, int B,
+                                  const void* kc, const void* vc, int t_max, const int32_t* lens,
+                                  const char* who) {
+  if (!b) return fail(LB_ERR_INVALID_ARG, "%s: NULL handle", who);
+  if (!x || !y || !kc || !vc || !lens) return fail(LB_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (B <= 0 || t_max <= 0) return fail(LB_ERR_INVALID_ARG, "%s: B and t_max must be positive", who);
+  if (x == y) return fail(LB_ERR_INVALID_ARG, "%s: y must not alias x", who);
+  if (!b->has_weights) return fail(LB_ERR_NO_WEIGHTS, "%s: set_weights was not called", who);
+  return LB_OK;
+}
+
+lb_status llama_block_prefill(llama_block* b, const void* x, void* y, int B, int T, void* k_cache,
+                              void* v_cache, int t_max, int32_t* cache_len, void* stream) {
+  lb_status st = check_cache_args(b, x, y, B, k_cache, v_cache, t_max, cache_len, "prefill");
+  if (st != LB_OK) return st;
+  if (T <= 0) return fail(LB_ERR_INVALID_ARG, "prefill: T must be positive");
+  if (T > t_max || T > b->max_pos)
+    return fail(LB_ERR_CACHE_FULL, "prefill: T=%d exceeds t_max=%d or max_pos=%d", T, t_max,
+                b->max_pos);
+  cudaStream_t s = (cudaStream_t)stream;
+  const int M = B * T;
+  size_t need = 0;
+  carve_prefill(b, nullptr, M, &need);
+  if ((st = ensure_ws(b, need)) != LB_OK) return st;
+  PrefillWs w = carve_prefill(b, b->ws, M, &need);
+  const int d = b->d, H = b->H, Hkv = b->Hkv, dh = b->dh, f = b->f;
+
+  if (b->dtype == kBF16) {
+    LB_CUDA(launch_resid_rmsnorm(kBF16, x, nullptr, 0, 0, nullptr, b->g1, w.h, M, d, b->eps, s));
+    GemmEpi e1;
+    e1.kind = kEpiQkvRope;
+    e1.T = T; e1.H = H; e1.Hkv = Hkv; e1.dh = dh; e1.t_max = t_max; e1.max_pos = b->max_pos;
+    e1.q_out = w.q; e1.k_cache = k_cache; e1.v_cache = v_cache;
+    e1.cos_t = b->cos_t; e1.sin_t = b->sin_t; e1.err = b->err;
+    LB_CUDA(launch_gemm_tc(w.h, b->w_qkv, M, b->n_qkv, d, 256, 1, e1, b->num_sms, s));
+    LB_CUDA(launch_attn_tc(w.q, k_cache, v_cache, w.o, B, T, T, H, Hkv, dh, t_max, b->err, s));
+    GemmEpi e2;
+    e2.kind = kEpiResid; e2.out = w.x1; e2.resid = x; e2.ldo = d; e2.err = b->err;
+    LB_CUDA(launch_gemm_tc(w.o, b->w_o, M, d, H * dh, 256, 1, e2, b->num_sms, s));
+    LB_CUDA(launch_resid_rmsnorm(kBF16, w.x1, nullptr, 0, 0, nullptr, b->g2, w.h, M, d, b->eps, s));
+    GemmEpi e3;
+    e3.kind = kEpiSwiGLU; e3.out = w.a; e3.ldo = f; e3.f = f; e3.err = b->err;
+    LB_CUDA(launch_gemm_tc(w.h, b->w_gu, M, b->n_gu, d, 256, 1, e3, b->num_sms, s));
+    GemmEpi e4;
+    e4.kind = kEpiResid; e4.out = y; e4.resid = w.x1; e4.ldo = d; e4.err = b->err;
+    LB_CUDA(launch_gemm_tc(w.a, b->w_d, M, d, f, 256, 1, e4, b->num_sms, s));
+  } else {
+    const float* X = (const float*)x;
+    LB_CUDA(launch_resid_rmsnorm(kF32, x, nullptr, 0, 0, nullptr, b->g1, w.h, M, d, b->eps, s));
+    LB_CUDA(launch_gemm_f32((const float*)w.h, (const float*)b->w_qkv, w.qkv32, nullptr, M,
+                            b->n_qkv, d, s));
+    LB_CUDA(launch_qkv_finish(kF32, w.qkv32, 1, 0, M, T, H, Hkv, dh, nullptr, b->cos_t, b->sin_t,
+                              b->max_pos, w.q, k_cache, v_cache, t_max, b->err, s));
+    LB_CUDA(launch_attn_f32((const float*)w.q, (const float*)k_cache, (const float*)v_cache,
+                            (float*)w.o, B, T, T, H, Hkv, dh, t_max, nullptr, s));
+    LB_CUDA(launch_gemm_f32((const float*)w.o, (const float*)b->w_o, (float*)w.x1, X, M, d,
+                            H * dh, s));
+    LB_CUDA(launch_resid_rmsnorm(kF32, w.x1, nullptr, 0, 0, nullptr, b->g2, w.h, M, d, b->eps, s));
+    LB_CUDA(launch_gemm_f32((const float*)w.h, (const float*)b->w_gu, w.gu32, nullptr, M, b->n_gu,
+                            d, s));
+    LB_CUDA(launch_silu_mul(kF32, w.gu32, 1, 0, M, f, b->n_gu, 0, w.a, s));
+    LB_CUDA(launch_gemm_f32((const float*)w.a, (const float*)b->w_d, (float*)y,
+                            (const float*)w.x1, M, d, f, s));
+  }
+  LB_CUDA(launch_set_lens(cache_len, B, T, s));
+  b->lens.assign(B, T);
+  return LB_OK;
+}
+
+lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void* k_cache,
+                             void* v_cache, int t_max, int32_t* cache_len, void* stream) {
+  lb_status st = check_cache_args(b, x, y, B, k_cache, v_cache, t_max, cache_len, "decode");
+  if (st != LB_OK) return st;
+  if ((int)b->lens.size() != B)
+    return fail(LB_ERR_INVALID_ARG,
+                "decode: the handle knows %d sequence lengths, B=%d (call prefill or set_lengths)",
+                (int)b->lens.size(), B);
+  for (int i = 0; i < B; ++i)
+    if (b->lens[i] < 0 || b->lens[i] + 1 > t_max || b->lens[i] >= b->max_pos)
+      return fail(LB_ERR_CACHE_FULL, "decode: sequence %d at length %d cannot grow (t_max=%d, max_pos=%d)",
+                  i, b->lens[i], t_max, b->max_pos);
+  cudaStream_t s = (cudaStream_t)stream;
+  size_t need = 0;
+  carve_decode(b, nullptr, B, t_max, &need);
+  if ((st = ensure_ws(b, need)) != LB_OK) return st;
+  DecodeWs w = carve_decode(b, b->ws, B, t_max, &need);
+  const int d = b->d, H = b->H, Hkv = b->Hkv, dh = b->dh, f = b->f;
+
+  if (b->dtype == kBF16) {
+    const int bn = B <= 32 ? 32 : B <= 64 ? 64 : B <= 128 ? 128 : 256;
+    LB_CUDA(launch_resid_rmsnorm(kBF16, x, nullptr, 0, 0, nullptr, b->g1, w.h, B, d, b->eps, s));
+    // Q|K|V: part[s][token][feature]
+    GemmEpi e;
+    e.kind = kEpiPartialT; e.out = w.part; e.err = b->err;
+    e.ldo = b->n_qkv; e.split_stride = (long long)B * b->n_qkv;
+    const int s1 = decode_split((b->n_qkv + 127) / 128, d);
+    LB_CUDA(launch_gemm_tc(b->w_qkv, w.h, b->n_qkv, B, d, bn, s1, e, b->num_sms, s));
+    const int s1e = gemm_effective_split(d, s1);
+    LB_CUDA(launch_qkv_finish(kBF16, w.part, s1e, e.split_stride, B, 1, H, Hkv, dh, cache_len,
+                              b->cos_t, b->sin_t, b->max_pos, w.q, k_cache, v_cache, t_max, b->err,
+                              s));
+    LB_CUDA(launch_attn_decode(w.q, k_cache, v_cache, w.o, w.attn_part, B, H, Hkv, dh, t_max,
+                               cache_len, b->err, s));
+    // o_proj, then X' = X + sum(partials) and h2 = RMSNorm(X') in one kernel
+    const int K2 = H * dh;
+    const int s2 = decode_split((d + 127) / 128, K2);
+    e.ldo = d; e.split_stride = (long long)B * d;
+    LB_CUDA(launch_gemm_tc(b->w_o, w.o, d, B, K2, bn, s2, e, b->num_sms, s));
+    const int s2e = gemm_effective_split(K2, s2);
+    LB_CUDA(launch_resid_rmsnorm(kBF16, x, w.part, s2e, e.split_stride, w.x1, b->g2, w.h, B, d,
+                                 b->eps, s));
+    // gate/up (packed rows), SiLU(g) * u
+    const int s3 = decode_split((b->n_gu + 127) / 128, d);
+    e.ldo = b->n_gu; e.split_stride = (long long)B * b->n_gu;
+    LB_CUDA(launch_gemm_tc(b->w_gu, w.h, b->n_gu, B, d, bn, s3, e, b->num_sms, s));
+    const int s3e = gemm_effective_split(d, s3);
+    LB_CUDA(launch_silu_mul(kBF16, w.part, s3e, e.split_stride, B, f, b->n_gu, 128, w.a, s));
+    // down, y = X' + sum(partials); cache_len += 1
+    const int s4 = decode_split((d + 127) / 128, f);
+    e.ldo = d; e.split_stride = (long long)B * d;
+    LB_CUDA(launch_gemm_tc(b->w_d, w.a, d, B, f, bn, s4, e, b->num_sms, s));
+    const int s4e = gemm_effective_split(f, s4);
+    LB_CUDA(launch_resid_add(kBF16, w.x1, w.part, s4e, e.split_stride, y, (long long)B * d,
+                             cache_len, B, 1, s));
+  } else {
+    const float* X = (const float*)x;
+    LB_CUDA(launch_resid_rmsnorm(kF32, x, nullptr, 0, 0, nullptr, b->g1, w.h, B, d, b->eps, s));
+    LB_CUDA(launch_gemm_f32((const float*)w.h, (const float*)b->w_qkv, w.part, nullptr, B,
+                            b->n_qkv, d, s));
+    LB_CUDA(launch_qkv_finish(kF32, w.part, 1, 0, B, 1, H, Hkv, dh, cache_len, b->cos_t, b->sin_t,
+                              b->max_pos, w.q, k_cache, v_cache, t_max, b->err, s));
+    LB_CUDA(launch_attn_f32((const float*)w.q, (const float*)k_cache, (const float*)v_cache,
+                            (float*)w.o, B, 1, 1, H, Hkv, dh, t_max, cache_len, s));
+    LB_CUDA(launch_gemm_f32((const float*)w.o, (const float*)b->w_o, (float*)w.x1, X, B, d,
+                            H * dh, s));
+    LB_CUDA(launch_resid_rmsnorm(kF32, w.x1, nullptr, 0, 0, nullptr, b->g2, w.h, B, d, b->eps, s));
+    LB_CUDA(launch_gemm_f32((const float*)w.h, (const float*)b->w_gu, w.part, nullptr, B, b->n_gu,
+                            d, s));
+    LB_CUDA(launch_silu_mul(kF32, w.part, 1, 0, B, f, b->n_gu, 0, w.a, s));
+    LB_CUDA(launch_gemm_f32((const float*)w.a, (const float*)b->w_d, (float*)y,
+                            (const float*)w.x1, B, d, f, s));
+    LB_CUDA(launch_resid_add(kF32, nullptr, nullptr, 0, 0, nullptr, 0, cache_len, B, 1, s));
+  }
+  for (int i = 0; i < B; ++i) b->lens[i] += 1;
+  return LB_OK;
+}
+
+static const char* describe_err(int code) {
+  if (code >= kErrWaitBase && code < kErrWaitBase + 0x100) return "a bounded device wait ran out";
+  return "a device-side bounds guard fired (cache index or RoPE position out of range)";
+}
+
+lb_status llama_block_sync_status(llama_block* b, void* stream) {
+  int* word = b ? b->err : standalone_err_word();
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return fail(LB_ERR_CUDA, "sync_status: %s", cudaGetErrorString(e));
+  if (!word) return fail(LB_ERR_CUDA, "sync_status: no error word");
+  int code = 0;
+  LB_CUDA(cudaMemcpy(&code, word, sizeof(int), cudaMemcpyDeviceToHost));
+  if (code == 0) return LB_OK;
+  LB_CUDA(cudaMemset(word, 0, sizeof(int)));
+  const bool wait = code >= kErrWaitBase && code < kErrWaitBase + 0x100;
+  return fail(wait ? LB_ERR_TIMEOUT : LB_ERR_CACHE_FULL, "device error 0x%x: %s", code,
+              describe_err(code));
+}
+
+lb_status llama_block_selftest_timeout(long long budget_ns, void* stream) {
+  if (budget_ns <= 0) return fail(LB_ERR_INVALID_ARG, "selftest_timeout: budget must be positive");
+  int* word = standalone_err_word();
+  if (!word) return fail(LB_ERR_CUDA, "selftest_timeout: no device");
+  LB_CUDA(launch_selftest_timeout(word, (unsigned long long)budget_ns, (cudaStream_t)stream));
+  return LB_OK;
+}
+
+// ------------------------------------------------------------------ standalone
+static lb_status check_dtype(lb_dtype dt, const char* who) {
+  if (dt != LB_F32 && dt != LB_BF16) return fail(LB_ERR_INVALID_ARG, "%s: bad dtype", who);
+  return LB_OK;
+}
+
+lb_status rmsnorm(const void* x, const void* g, void* y, int rows, int d, float eps,
+                  lb_dtype dtype, void* stream) {
+  if (check_dtype(dtype, "rmsnorm") != LB_OK) return LB_ERR_INVALID_ARG;
+  if (!x || !g || !y) return fail(LB_ERR_INVALID_ARG, "rmsnorm: NULL pointer");
+  if (rows < 0 || d <= 0 || !(eps > 0.f)) return fail(LB_ERR_INVALID_ARG, "rmsnorm: bad size");
+  if (d % 8 != 0 || d > 8192)
+    return fail(LB_ERR_UNSUPPORTED, "rmsnorm: d must be a multiple of 8 and <= 8192");
+  LB_CUDA(launch_resid_rmsnorm(dtype, x, nullptr, 0, 0, nullptr, g, y, rows, d, eps,
+                               (cudaStream_t)stream));
+  return LB_OK;
+}
+
+lb_status rope_apply(void* x, const int32_t* pos, int B, int T, int n_heads, int head_dim,
+                     float base, lb_dtype dtype, void* stream) {
+  if (check_dtype(dtype, "rope_apply") != LB_OK) return LB_ERR_INVALID_ARG;
+  if (!x || !pos) return fail(LB_ERR_INVALID_ARG, "rope_apply: NULL pointer");
+  if (B < 0 || T < 0 || n_heads <= 0 || head_dim <= 0 || head_dim % 2 || !(base > 0.f))
+    return fail(LB_ERR_INVALID_ARG, "rope_apply: bad size");
+  LB_CUDA(launch_rope_apply(dtype, x, pos, B, T, n_heads, head_dim, (double)base,
+                            (cudaStream_t)stream));
+  return LB_OK;
+}
+
+lb_status causal_attn(const void* q, const void* k, const void* v, void* o, int B, int Tq, int Tk,
+                      int n_heads, int n_kv_heads, int head_dim, int k_stride_T, lb_dtype dtype,
+                      void* stream) {
+  if (check_dtype(dtype, "causal_attn") != LB_OK) return LB_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o) return fail(LB_ERR_INVALID_ARG, "causal_attn: NULL pointer");
+  if (B < 0 || Tq < 1 || Tk < Tq || k_stride_T < Tk || n_heads <= 0 || n_kv_heads <= 0)
+    return fail(LB_ERR_INVALID_ARG, "causal_attn: need 1 <= Tq <= Tk <= k_stride_T");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(LB_ERR_UNSUPPORTED, "causal_attn: head_dim %d not in {64,128}", head_dim);
+  if (n_heads % n_kv_heads) return fail(LB_ERR_UNSUPPORTED, "causal_attn: n_heads %% n_kv_heads");
+  cudaStream_t s = (cudaStream_t)stream;
+  if (dtype == LB_BF16) {
+    int* err = standalone_err_word();
+    LB_CUDA(launch_attn_tc(q, k, v, o, B, Tq, Tk, n_heads, n_kv_heads, head_dim, k_stride_T, err, s));
+  } else {
+    LB_CUDA(launch_attn_f32((const float*)q, (const float*)k, (const float*)v, (float*)o, B, Tq, Tk,
+                            n_heads, n_kv_heads, head_dim, k_stride_T, nullptr, s));
+  }
+  return LB_OK;
+}
+
+lb_status swiglu_mlp(const void* h, const void* w_gate, const void* w_up, const void* w_down,
+                     void* y, int M, int d, int f, lb_dtype dtype, void* stream) {
+  if (check_dtype(dtype, "swiglu_mlp") != LB_OK) return LB_ERR_INVALID_ARG;
+  if (!h || !w_gate || !w_up || !w_down || !y) return fail(LB_ERR_INVALID_ARG, "swiglu_mlp: NULL pointer");
+  if (M < 0 || d <= 0 || f <= 0) return fail(LB_ERR_INVALID_ARG, "swiglu_mlp: bad size");
+  if (dtype == LB_BF16 && (d % 64 || f % 8))
+    return fail(LB_ERR_UNSUPPORTED, "swiglu_mlp: bf16 needs d %% 64 == 0 and f %% 8 == 0");
+  if (M == 0) return LB_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t es = dtype == LB_F32 ? 4 : 2;
+  const int f_pad = dtype == LB_BF16 ? (f + 127) / 128 * 128 : f;
+  const int n_gu = 2 * f_pad;
+  char* tmp = nullptr;
+  const size_t wbytes = align_up((size_t)n_gu * d * es, 256);
+  const size_t abytes = align_up((size_t)M * f_pad * es, 256);
+  const size_t gbytes = dtype == LB_F32 ? (size_t)M * n_gu * 4 : 0;
+  LB_CUDA(cudaMallocAsync((void**)&tmp, wbytes + abytes + gbytes, s));
+  lb_status st = LB_OK;
+  auto run = [&]() -> lb_status {
+    LB_CUDA(cudaMemsetAsync(tmp, 0, wbytes, s));
+    if (dtype == LB_F32) {
+      LB_CUDA(cudaMemcpyAsync(tmp, w_gate, (size_t)f * d * es, cudaMemcpyDeviceToDevice, s));
+      LB_CUDA(cudaMemcpyAsync(tmp + (size_t)f * d * es, w_up, (size_t)f * d * es,
+                              cudaMemcpyDeviceToDevice, s));
+      float* gu = (float*)(tmp + wbytes + abytes);
+      LB_CUDA(launch_gemm_f32((const float*)h, (const float*)tmp, gu, nullptr, M, n_gu, d, s));
+      LB_CUDA(launch_silu_mul(kF32, gu, 1, 0, M, f, n_gu, 0, tmp + wbytes, s));
+      LB_CUDA(launch_gemm_f32((const float*)(tmp + wbytes), (const float*)w_down, (float*)y,
+                              nullptr, M, d, f, s));
+    } else {
+      const size_t blk = 128 * (size_t)d * es;
+      const int full = f / 128, rem = f - full * 128;
+      if (full > 0) {
+        LB_CUDA(cudaMemcpy2DAsync(tmp, 2 * blk, w_gate, blk, blk, full, cudaMemcpyDeviceToDevice, s));
+        LB_CUDA(cudaMemcpy2DAsync(tmp + blk, 2 * blk, w_up, blk, blk, full,
+                                  cudaMemcpyDeviceToDevice, s));
+      }
+      if (rem > 0) {
+        const size_t src = (size_t)full * blk;
+        LB_CUDA(cudaMemcpyAsync(tmp + 2 * src, (const char*)w_gate + src, rem * d * es,
+                                cudaMemcpyDeviceToDevice, s));
+        LB_CUDA(cudaMemcpyAsync(tmp + 2 * src + blk, (const char*)w_up + src, rem * d * es,
+                                cudaMemcpyDeviceToDevice, s));
+      }
+      const int nsm = num_sms_of_current_device();
+      GemmEpi e3;
+      e3.kind = kEpiSwiGLU; e3.out = tmp + wbytes; e3.ldo = f; e3.f = f;
+      e3.err = standalone_err_word();
+      LB_CUDA(launch_gemm_tc(h, tmp, M, n_gu, d, 256, 1, e3, nsm, s));
+      GemmEpi e4;
+      e4.kind = kEpiStore; e4.out = y; e4.ldo = d; e4.err = e3.err;
+      LB_CUDA(launch_gemm_tc(tmp + wbytes, w_down, M, d, f, 256, 1, e4, nsm, s));
+    }
+    return LB_OK;
+  };
+  st = run();
+  cudaFreeAsync(tmp, s);
+  return st;
+}
+
+}  // extern "C"

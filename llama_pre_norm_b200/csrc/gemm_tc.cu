@@ -1,0 +1,427 @@
+// gemm_tc.cu — bf16 GEMM on the 5th-generation tensor cores (tcgen05 + TMEM),
+// fed by TMA, for the four dense contractions of the block (the fused Q|K|V
+// projection, o_proj, the fused gate/up projection and down_proj of the
+// LlamaAttention / LlamaMLP modules, LMDrive page §2.3–§2.4).
+//
+//   D[M,N] = A[M,K] · B[N,K]^T        (both operands K-major, fp32 accumulation)
+//
+// Structure (one persistent CTA per SM, 192 threads):
+//   warp 0      TMA producer: 128x64 A and BNx64 B boxes (128-byte swizzle) into
+//               a STAGES-deep shared-memory ring, completion via mbarrier tx counts;
+//   warp 1      allocates TMEM, and one thread issues tcgen05.mma (M=128, N=BN,
+//               K=16 per instruction) into one of two TMEM accumulators, then
+//               tcgen05.commit frees the smem slot / publishes the accumulator;
+//   warps 2..5  epilogue: tcgen05.ld (each warp reads its 32-lane TMEM quarter,
+//               one output row per thread), fused op, vectorised global stores.
+// Two accumulators let the epilogue of tile i overlap the main loop of tile i+1.
+//
+// Fused epilogues: residual add (o_proj, down_proj: the two residual adds of the
+// pre-norm layer, §2.5), SiLU(gate)*up (gate/up rows interleaved in blocks of
+// 128 so one 256-wide tile holds matching gate and up columns, §2.4), RoPE on Q
+// and K with the scatter of Q into [B,H,T,dh] and K/V into the KV cache (§2.2,
+// §2.3), and an fp32 split-K partial store for the swap-AB decode GEMMs.
+#include "common.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace lb {
+
+constexpr int kBM = 128, kBK = 64;
+constexpr int kGemmThreads = 192;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+};
+
+struct Unit {
+  int mt, nt, s, kb0, kb1;
+};
+
+__device__ __forceinline__ Unit decode_unit(int u, int num_m, int num_n, int KB, int kb_per) {
+  Unit r;
+  const int mn = num_m * num_n;
+  r.s = u / mn;
+  const int rem = u - r.s * mn;
+  r.mt = rem % num_m;  // m fastest: concurrent CTAs share one weight (B) tile
+  r.nt = rem / num_m;
+  r.kb0 = r.s * kb_per;
+  r.kb1 = min(KB, r.kb0 + kb_per);
+  return r;
+}
+
+// ------------------------------------------------------------------ epilogues
+// Store 32 consecutive values of one output row at columns [n, n+32) of a row
+// with `ncols` columns: vectorised when the whole run is in range, else only
+// the in-range elements (ragged last tile).
+__device__ __forceinline__ void store_row32(bf16* row, int n, int ncols, const float (&v)[32]) {
+  if (n + 32 <= ncols) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float t[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) t[i] = v[q * 8 + i];
+      store8(row + n + q * 8, t);
+    }
+  } else {
+    for (int i = 0; i < 32 && n + i < ncols; ++i) row[n + i] = __float2bfloat16_rn(v[i]);
+  }
+}
+
+template <int BN>
+__device__ __forceinline__ void epi_store_resid(uint32_t tb, int m, int nt, int M, int N,
+                                                const GemmEpi& e, bool with_resid) {
+  bf16* out = reinterpret_cast<bf16*>(e.out);
+  const bf16* res = reinterpret_cast<const bf16*>(e.resid);
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    float v[32];
+    tmem_ld32(tb + c * 32, v);
+    tmem_wait_ld();
+    const int n = nt * BN + c * 32;
+    if (m < M && n < N) {
+      const long long o = (long long)m * e.ldo;
+      if (with_resid) {
+        if (n + 32 <= N) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float r[8];
+            load8(res + o + n + q * 8, r);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[q * 8 + i] += r[i];
+          }
+        } else {
+          for (int i = 0; i < 32 && n + i < N; ++i) v[i] += __bfloat162float(res[o + n + i]);
+        }
+      }
+      store_row32(out + o, n, N, v);
+    }
+  }
+}
+
+// Tile columns [0,128) are gate rows 128*nt.., [128,256) the matching up rows.
+__device__ __forceinline__ void epi_swiglu(uint32_t tb, int m, int nt, int M, int f,
+                                           const GemmEpi& e) {
+  bf16* out = reinterpret_cast<bf16*>(e.out);
+#pragma unroll 1
+  for (int j = 0; j < 4; ++j) {
+    float g[32], u[32];
+    tmem_ld32(tb + j * 32, g);
+    tmem_ld32(tb + 128 + j * 32, u);
+    tmem_wait_ld();
+    const int col = nt * 128 + j * 32;
+    if (m < M && col < f) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
+      store_row32(out + (long long)m * e.ldo, col, f, g);
+    }
+  }
+}
+
+// Columns of the fused projection: Q heads [0, H*dh), K heads, then V heads.
+// Each thread owns token row m = b*T + t at position t; RoPE pairs column i with
+// i + dh/2 of the same head (rotate_half), both held by this thread.
+template <int BN>
+__device__ __forceinline__ void epi_qkv_rope(uint32_t tb, int m, int nt, int M, int N,
+                                             const GemmEpi& e) {
+  const int dh = e.dh, half = dh >> 1;
+  const int b = m / e.T, t = m - (m / e.T) * e.T;
+  const int pos = t;
+  const bool row_ok = m < M;
+  bool pos_ok = pos < e.max_pos && pos < e.t_max;
+  if (row_ok && !pos_ok) latch_error(e.err, kErrCacheBounds);
+#pragma unroll 1
+  for (int hh = 0; hh < BN / dh; ++hh) {
+    const int gcol = nt * BN + hh * dh;
+    if (gcol >= N) break;  // uniform across the warp
+    const int hq = gcol / dh;
+    bf16* dst;
+    bool rotate = true;
+    if (hq < e.H) {
+      dst = reinterpret_cast<bf16*>(e.q_out) + (((long long)b * e.H + hq) * e.T + t) * dh;
+    } else if (hq < e.H + e.Hkv) {
+      dst = reinterpret_cast<bf16*>(e.k_cache) +
+            (((long long)b * e.Hkv + (hq - e.H)) * e.t_max + pos) * dh;
+    } else {
+      dst = reinterpret_cast<bf16*>(e.v_cache) +
+            (((long long)b * e.Hkv + (hq - e.H - e.Hkv)) * e.t_max + pos) * dh;
+      rotate = false;
+    }
+    const bool store = row_ok && pos_ok;
+    if (rotate) {
+#pragma unroll 1
+      for (int j = 0; j < half / 32; ++j) {
+        float x1[32], x2[32];
+        tmem_ld32(tb + hh * dh + j * 32, x1);
+        tmem_ld32(tb + hh * dh + half + j * 32, x2);
+        tmem_wait_ld();
+        if (store) {
+          const float* ct = e.cos_t + (long long)pos * half + j * 32;
+          const float* st = e.sin_t + (long long)pos * half + j * 32;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float c[8], s[8], o1[8], o2[8];
+            load8(ct + q * 8, c);
+            load8(st + q * 8, s);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float a = x1[q * 8 + i], bb = x2[q * 8 + i];
+              o1[i] = a * c[i] - bb * s[i];
+              o2[i] = bb * c[i] + a * s[i];
+            }
+            store8(dst + j * 32 + q * 8, o1);
+            store8(dst + half + j * 32 + q * 8, o2);
+          }
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int j = 0; j < dh / 32; ++j) {
+        float x[32];
+        tmem_ld32(tb + hh * dh + j * 32, x);
+        tmem_wait_ld();
+        if (store) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = x[q * 8 + i];
+            store8(dst + j * 32 + q * 8, o);
+          }
+        }
+      }
+    }
+  }
+}
+
+// Swap-AB decode: rows are weight rows (output features), columns are tokens.
+// part[s][token][row] = acc, so that a warp's 32 lanes write 32 consecutive floats.
+template <int BN>
+__device__ __forceinline__ void epi_partial_t(uint32_t tb, int row, int nt, int s, int M, int N,
+                                              const GemmEpi& e) {
+  float* part = reinterpret_cast<float*>(e.out) + (long long)s * e.split_stride;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    float v[32];
+    tmem_ld32(tb + c * 32, v);
+    tmem_wait_ld();
+    if (row < M) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int tok = nt * BN + c * 32 + i;
+        if (tok < N) part[(long long)tok * e.ldo + row] = v[i];
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   int M, int N, int K, int kb_per, int n_split, GemmEpi epi) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::STAGES;
+  uint64_t* tfull = bars + 2 * C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_m = (M + kBM - 1) / kBM, num_n = (N + BN - 1) / BN;
+  const int KB = (K + kBK - 1) / kBK;
+  const int units = num_m * num_n * n_split;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      uint32_t stage = 0, phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(u, num_m, num_n, KB, kb_per);
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, epi.err, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * kBK, w.mt * kBM);
+          tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * kBK, w.nt * BN);
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Every load issued must land before the CTA may exit.
+      const long long first = issued > C::STAGES ? issued - C::STAGES : 0;
+      for (long long i = first; i < issued; ++i)
+        mbar_wait(&full[i % C::STAGES], (uint32_t)((i / C::STAGES) & 1), epi.err, 6);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      constexpr uint32_t idesc = umma_idesc_bf16(kBM, BN, 0, 0);
+      uint32_t stage = 0, phase = 0;
+      int t = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++t) {
+        const Unit w = decode_unit(u, num_m, num_n, KB, kb_per);
+        const int acc = t & 1;
+        if (!mbar_wait(&tempty[acc], ((t >> 1) & 1) ^ 1, epi.err, 2)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, epi.err, 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t ad = umma_desc_sw128(a0 + k * 32, 16, 1024);
+            const uint64_t bd = umma_desc_sw128(b0 + k * 32, 16, 1024);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+      }
+      // All issued MMAs must complete before TMEM is released.
+      umma_commit(drain);
+      mbar_wait(drain, 0, epi.err, 4);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5)
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int row_in_tile = quarter * 32 + lane;
+    int t = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++t) {
+      const Unit w = decode_unit(u, num_m, num_n, KB, kb_per);
+      const int acc = t & 1;
+      if (!mbar_wait(&tfull[acc], (t >> 1) & 1, epi.err, 5)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      const int m = w.mt * kBM + row_in_tile;
+      if constexpr (EPI == kEpiStore) {
+        epi_store_resid<BN>(tb, m, w.nt, M, N, epi, false);
+      } else if constexpr (EPI == kEpiResid) {
+        epi_store_resid<BN>(tb, m, w.nt, M, N, epi, true);
+      } else if constexpr (EPI == kEpiSwiGLU) {
+        epi_swiglu(tb, m, w.nt, M, epi.f, epi);
+      } else if constexpr (EPI == kEpiQkvRope) {
+        epi_qkv_rope<BN>(tb, m, w.nt, M, N, epi);
+      } else {
+        epi_partial_t<BN>(tb, m, w.nt, w.s, M, N, epi);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+template <int BN, int EPI>
+static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
+                       int kb_per, int n_split, const GemmEpi& epi, int grid, cudaStream_t s) {
+  using C = GemmCfg<BN>;
+  auto kern = gemm_tc_kernel<BN, EPI>;
+  static bool attr_set = false;  // per instantiation; the attribute is per device function
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<grid, kGemmThreads, C::SMEM, s>>>(ta, tb, M, N, K, kb_per, n_split, epi);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, int BN, int n_split,
+                           const GemmEpi& epi, int num_sms, cudaStream_t s) {
+  if (M <= 0 || N <= 0 || K <= 0) return cudaSuccess;
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d_bf16(&ta, A, (uint64_t)M, (uint64_t)K, kBM)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d_bf16(&tb, B, (uint64_t)N, (uint64_t)K, (uint32_t)BN))
+    return cudaErrorInvalidValue;
+  const int KB = (K + kBK - 1) / kBK;
+  n_split = gemm_effective_split(K, n_split);
+  const int kb_per = (KB + n_split - 1) / n_split;
+  const long long units =
+      (long long)((M + kBM - 1) / kBM) * ((N + BN - 1) / BN) * (long long)n_split;
+  const int grid = (int)std::min<long long>(units, num_sms);
+  switch (epi.kind) {
+    case kEpiStore:
+      if (BN == 256) return run<256, kEpiStore>(ta, tb, M, N, K, kb_per, n_split, epi, grid, s);
+      if (BN == 128) return run<128, kEpiStore>(ta, tb, M, N, K, kb_per, n_split, epi, grid, s);
+      break;
+    case kEpiResid:
+      if (BN == 256) return run<256, kEpiResid>(ta, tb, M, N, K, kb_per, n_split, epi, grid, s);
+      if (BN == 128) return run<128, kEpiResid>(ta, tb, M, N, K, kb_per, n_split, epi, grid, s);
+      break;
+    case kEpiSwiGLU:
+      if (BN == 256) return run<256, kEpiSwiGLU>(ta, tb, M, N, K, kb_per, n_split, epi, grid, s);
+      break;
+    case kEpiQkvRope:
+      if (BN == 256) return run<256, kEpiQkvRope>(ta, tb, M, N, K, kb_per, n_split, epi, grid, s);
+      break;
+    case kEpiPartialT:
+      if (BN == 32) return run<32, kEpiPartialT>(ta, tb, M, N, K, kb_per, n_split, epi, grid, s);
+      if (BN == 64) return run<64, kEpiPartialT>(ta, tb, M, N, K, kb_per, n_split, epi, grid, s);
+      if (BN == 128) return run<128, kEpiPartialT>(ta, tb, M, N, K, kb_per, n_split, epi, grid, s);
+      if (BN == 256) return run<256, kEpiPartialT>(ta, tb, M, N, K, kb_per, n_split, epi, grid, s);
+      break;
+  }
+  return cudaErrorInvalidConfiguration;
+}
+
+}  // namespace lb

@@ -1,0 +1,116 @@
+// internal.h — launch interface between the C-ABI layer (capi.cu) and the kernels.
+// Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+namespace lb {
+
+enum { kF32 = 0, kBF16 = 1 };
+
+// Codes latched into a device error word (first error wins).
+enum : int {
+  kErrNone = 0,
+  kErrWaitBase = 0x100,     // + wait-site id: a bounded wait ran out
+  kErrCacheBounds = 0x200,  // a KV-cache index outside [0, t_max)
+  kErrPosBounds = 0x201,    // a RoPE position outside the table
+};
+
+// Split-K count actually used for K and a requested count: every split non-empty.
+inline int gemm_effective_split(int K, int n_split) {
+  const int KB = (K + 63) / 64;
+  n_split = std::max(1, std::min(n_split, KB));
+  const int per = (KB + n_split - 1) / n_split;
+  return (KB + per - 1) / per;
+}
+
+// ----------------------------------------------------------- norm_fuse.cu
+cudaError_t launch_resid_rmsnorm(int dtype, const void* x, const float* partial, int n_split,
+                                 long long split_stride, void* x_out, const void* g, void* y,
+                                 int rows, int d, float eps, cudaStream_t s);
+cudaError_t launch_qkv_finish(int dtype, const float* qkv, int n_split, long long split_stride,
+                              int M, int T, int H, int Hkv, int dh, const int* pos_base,
+                              const float* cos_t, const float* sin_t, int max_pos, void* q_out,
+                              void* k_cache, void* v_cache, int t_max, int* err, cudaStream_t s);
+cudaError_t launch_silu_mul(int dtype, const float* gu, int n_split, long long split_stride, int M,
+                            int f, int n_packed, int block, void* a, cudaStream_t s);
+cudaError_t launch_resid_add(int dtype, const void* resid, const float* part, int n_split,
+                             long long split_stride, void* out, long long total, int* lens, int B,
+                             int len_inc, cudaStream_t s);
+cudaError_t launch_set_lens(int* lens, int B, int value, cudaStream_t s);
+cudaError_t launch_rope_apply(int dtype, void* x, const int* pos, int B, int T, int H, int dh,
+                              double base, cudaStream_t s);
+cudaError_t launch_selftest_timeout(int* err, unsigned long long budget_ns, cudaStream_t s);
+
+// ----------------------------------------------------------- simt_f32.cu (fp32 path)
+// C[M,N] = A[M,K] B[N,K]^T (+ resid[M,N]); all fp32 row-major.
+cudaError_t launch_gemm_f32(const float* A, const float* B, float* C, const float* resid, int M,
+                            int N, int K, cudaStream_t s);
+// Causal attention, fp32. q [B,H,Tq,dh]; k,v [B,Hkv,k_stride,dh]; o [B,Tq,H*dh].
+// kv_len NULL: Tk keys, query i at Tk-Tq+i. kv_len[b] given: Tk_b = kv_len[b] + 1.
+cudaError_t launch_attn_f32(const float* q, const float* k, const float* v, float* o, int B,
+                            int Tq, int Tk, int H, int Hkv, int dh, int k_stride,
+                            const int* kv_len, cudaStream_t s);
+
+// ----------------------------------------------------------- gemm_tc.cu (bf16 tcgen05)
+enum EpiKind {
+  kEpiStore = 0,     // out[m][n] = bf16(acc)
+  kEpiResid = 1,     // out[m][n] = bf16(resid[m][n] + acc)
+  kEpiSwiGLU = 2,    // tile = [gate 128 | up 128] -> a[m][nt*128 + j] = bf16(silu(g)*u)
+  kEpiQkvRope = 3,   // RoPE on Q/K heads, scatter Q to [B,H,T,dh], K/V into the cache
+  kEpiPartialT = 4,  // swap-AB split-K: part[split][col][row] = acc (fp32)
+};
+
+struct GemmEpi {
+  int kind = kEpiStore;
+  void* out = nullptr;          // bf16 output / partial fp32 buffer
+  const void* resid = nullptr;  // bf16 residual [M, N]
+  long long ldo = 0;            // row stride of out / resid (elements)
+  long long split_stride = 0;   // kEpiPartialT: elements between split slabs
+  // kEpiQkvRope
+  int f = 0;                    // kEpiSwiGLU: number of output columns (intermediate size)
+  int T = 1, H = 0, Hkv = 0, dh = 128, t_max = 0, max_pos = 0;
+  void* q_out = nullptr;
+  void* k_cache = nullptr;
+  void* v_cache = nullptr;
+  const float* cos_t = nullptr;
+  const float* sin_t = nullptr;
+  int* err = nullptr;
+};
+
+// D[M,N] = A[M,K] · B[N,K]^T, bf16 operands (K-major, row stride K), fp32 accumulation in
+// TMEM. BN selects the N tile (256 / 128 / 32). n_split > 1 splits K (kEpiPartialT only).
+cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, int BN, int n_split,
+                           const GemmEpi& epi, int num_sms, cudaStream_t s);
+
+// ----------------------------------------------------------- attn_tc.cu (bf16 tcgen05)
+// Causal flash attention. q [B,H,Tq,dh]; k,v [B,Hkv,k_stride,dh]; o [B,Tq,H*dh].
+cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, int B, int Tq,
+                           int Tk, int H, int Hkv, int dh, int k_stride, int* err,
+                           cudaStream_t s);
+
+// ----------------------------------------------------------- attn_decode.cu (bf16)
+// Split-KV decode attention: one query per (b, h) at position kv_len[b], keys
+// 0..kv_len[b] (the new key already appended). q [B,H,dh]; k,v [B,Hkv,k_stride,dh];
+// o [B, H*dh]. `part` holds B*H*max_chunks*(dh+2) floats.
+int decode_attn_chunks(int k_stride);
+cudaError_t launch_attn_decode(const void* q, const void* k, const void* v, void* o, float* part,
+                               int B, int H, int Hkv, int dh, int k_stride, const int* kv_len,
+                               int* err, cudaStream_t s);
+
+// ----------------------------------------------------------- tensor maps
+// Encode a 2D bf16 tensor map over a row-major [rows, cols] matrix with a
+// box of [box_rows, 64 cols] and 128-byte swizzle.
+bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows);
+// 3D bf16 tensor map over [planes, rows, cols] (cols contiguous, rows `cols` apart,
+// planes `plane_stride` elements apart), box [1, box_rows, 64], 128-byte swizzle.
+// Rows >= `rows` read as zero.
+bool make_tmap_3d_bf16(CUtensorMap* m, const void* base, uint64_t planes, uint64_t rows,
+                       uint64_t cols, uint64_t plane_stride, uint32_t box_rows);
+
+}  // namespace lb

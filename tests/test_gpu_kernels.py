@@ -1,0 +1,126 @@
+"""GPU parity of the standalone entry points against the fp64 oracle.
+
+Each test feeds the same seeded inputs (rounded to the compute dtype) to the
+C ABI (through the ctypes binding) and to ``oracle/``, and compares element by
+element: fp32 within 1e-4 relative, bf16 within 2e-2 per-row max-norm. Sizes
+span several tiles with ragged tails."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import block as ob
+from synth import make_tensor
+from tests.helpers import BF16_TOL, F32_TOL, as_np, cuda, rel_err_floor, row_err
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import llama_pre_norm_b200 as lb
+
+
+def _tol(dt):
+    return F32_TOL if dt == torch.float32 else BF16_TOL
+
+
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("rows,d", [(1, 256), (7, 4096), (33, 5120), (5, 8192), (3, 8)])
+def test_rmsnorm(dt, rows, d):
+    x = make_tensor((rows, d), 100 + d, dt, std=2.0)
+    g = make_tensor((d,), 200 + d, dt, std=0.1, mean=1.0)
+    y = torch.empty_like(x, device="cuda")
+    lb.rmsnorm(cuda(x), cuda(g), y, 1e-6)
+    lb.llama_block_sync_status()
+    want = ob.rmsnorm(x, g, 1e-6)
+    assert row_err(y, want) <= _tol(dt)
+    if dt == torch.float32:
+        assert rel_err_floor(y, want) <= F32_TOL
+
+
+def test_rmsnorm_zero_rows_is_noop():
+    x = torch.zeros(0, 64, device="cuda")
+    lb.rmsnorm(x, torch.ones(64, device="cuda"), torch.zeros(0, 64, device="cuda"), 1e-6)
+    lb.llama_block_sync_status()
+
+
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dh", [64, 128])
+def test_rope_apply(dt, dh):
+    B, H, T = 2, 3, 37
+    x = make_tensor((B, H, T, dh), 300 + dh, dt)
+    pos = torch.randint(0, 5000, (B, T), generator=torch.Generator().manual_seed(7), dtype=torch.int32)
+    xg = cuda(x)
+    lb.rope_apply(xg, cuda(pos), 10000.0)
+    lb.llama_block_sync_status()
+    want = ob.apply_rope(x, pos.numpy().astype(np.float64)[:, None, :], 10000.0)
+    assert row_err(xg, want) <= _tol(dt)
+    if dt == torch.float32:
+        assert rel_err_floor(xg, want) <= F32_TOL
+
+
+ATTN_CASES = [
+    # B, H, Hkv, Tq, Tk, k_stride, dh
+    (1, 4, 4, 64, 64, 64, 64),        # tiny, single partial tile
+    (2, 4, 2, 300, 300, 320, 128),    # GQA, 3 query tiles, ragged tail
+    (1, 16, 2, 256, 256, 256, 128),   # n_rep = 8
+    (2, 2, 2, 130, 400, 512, 64),     # queries at an offset (chunked prefill)
+    (3, 2, 1, 1, 513, 600, 128),      # a single decode-like query per sequence
+    (1, 2, 2, 384, 384, 384, 128),    # exact tiles
+]
+
+
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("case", ATTN_CASES)
+def test_causal_attn(dt, case):
+    B, H, Hkv, Tq, Tk, ks, dh = case
+    q = make_tensor((B, H, Tq, dh), 400, dt)
+    k = make_tensor((B, Hkv, ks, dh), 401, dt)
+    v = make_tensor((B, Hkv, ks, dh), 402, dt)
+    kg, vg = cuda(k), cuda(v)
+    if ks > Tk:  # rows beyond Tk must never be read into the result
+        kg[:, :, Tk:] = float("nan")
+        vg[:, :, Tk:] = float("nan")
+    o = torch.empty(B, Tq, H * dh, dtype=dt, device="cuda")
+    lb.causal_attn(cuda(q), kg, vg, o, Tk=Tk)
+    lb.llama_block_sync_status()
+    want = ob.causal_attention(q, k[:, :, :Tk], v[:, :, :Tk])  # [B,H,Tq,dh]
+    want = want.transpose(0, 2, 1, 3).reshape(B, Tq, H * dh)
+    got = as_np(o).reshape(B, Tq, H, dh)
+    assert row_err(got, want.reshape(B, Tq, H, dh)) <= _tol(dt)
+    if dt == torch.float32:
+        assert rel_err_floor(got, want.reshape(B, Tq, H, dh)) <= F32_TOL
+
+
+@pytest.mark.parametrize("dt,M,d,f", [
+    (torch.float32, 17, 256, 688),
+    (torch.bfloat16, 300, 512, 1000),   # ragged M, f not a multiple of 128
+    (torch.bfloat16, 256, 1024, 2816),  # exact tiles
+    (torch.bfloat16, 5, 512, 384),
+])
+def test_swiglu_mlp(dt, M, d, f):
+    h = make_tensor((M, d), 500, dt)
+    wg = make_tensor((f, d), 501, dt, std=0.05)
+    wu = make_tensor((f, d), 502, dt, std=0.05)
+    wd = make_tensor((d, f), 503, dt, std=0.05)
+    y = torch.empty(M, d, dtype=dt, device="cuda")
+    lb.swiglu_mlp(cuda(h), cuda(wg), cuda(wu), cuda(wd), y)
+    lb.llama_block_sync_status()
+    want = ob.swiglu_mlp(h, wg, wu, wd)
+    assert row_err(y, want) <= _tol(dt)
+    if dt == torch.float32:
+        assert rel_err_floor(y, want) <= F32_TOL
+
+
+def test_bounded_wait_times_out_cleanly():
+    """A wait on a barrier nothing completes gives up after its budget, latches
+    the error word, and the context stays usable."""
+    lb.llama_block_selftest_timeout(50_000_000)  # 50 ms
+    with pytest.raises(lb.LlamaBlockError) as ei:
+        lb.llama_block_sync_status()
+    assert ei.value.name == "LB_ERR_TIMEOUT"
+    lb.llama_block_sync_status()  # cleared
+    x = torch.ones(2, 64, device="cuda")
+    y = torch.empty_like(x)
+    lb.rmsnorm(x, torch.ones(64, device="cuda"), y, 1e-6)
+    lb.llama_block_sync_status()
+    assert torch.allclose(y, torch.ones_like(y), atol=1e-5)

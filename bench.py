@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 LLaMA pre-norm decoder block.
+
+Headline: prefill of the LLaMA-7B-shaped block (bf16, d=4096, 32 heads, head_dim
+128, f=11008, B=1, T=2048) in tokens/s, with the fraction of dense BF16 tensor
+peak it reaches; beside it, the KV-cache decode step of the same block (B=32,
+cache 4096 -> 4224 over 128 steps) in HBM GB/s.
+
+One step = one prefill of the whole block (RMSNorm, fused QKV GEMM with RoPE and
+the KV-cache scatter, causal attention, o_proj + residual, RMSNorm, gate/up GEMM
+with SiLU*up, down_proj + residual) over the synthetic 2048-token input, called
+through the C ABI. Inputs are resident in HBM; L2 is flushed (256 MB write)
+before every timed step; each step is timed with CUDA events on the library's
+stream. Multi-GPU runs are independent replicas (one process per GPU, no
+data-path collective): value = all ranks' tokens / the slowest rank's time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm of this
+workload) on a bounded sample of the same prefill.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "7B-shape block prefill tokens/s & % BF16 peak; decode-step HBM GB/s"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+CPU_SAMPLE_T = 2048  # tokens of the 7B prefill the CPU oracle evaluates per sample (the full T)
+
+# DRAM traffic per launch of the dominant kernels from ncu captures (see
+# profiles/); None until a capture of the current kernel exists.
+NCU_TRAFFIC_BYTES = {
+    "gate_up_swiglu_gemm": None,
+    "attention_decode": None,
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=128)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks() -> dict:
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ workload accounting
+def prefill_flops(cfg) -> dict:
+    """Algorithmic FLOPs of one prefill: 2MNK per GEMM, causal attention pairs only."""
+    M = cfg.B * cfg.T
+    d, f, H, Hkv, dh = cfg.d, cfg.f, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    qkv = 2 * M * (H + 2 * Hkv) * dh * d
+    o = 2 * M * d * H * dh
+    gu = 2 * M * 2 * f * d
+    down = 2 * M * d * f
+    pairs = cfg.B * cfg.T * (cfg.T + 1) // 2
+    attn = 2 * 2 * pairs * dh * H  # QK^T and PV
+    return {"qkv": qkv, "o": o, "gate_up": gu, "down": down, "attn": attn,
+            "total": qkv + o + gu + down + attn}
+
+
+def decode_bytes(cfg, L: int) -> int:
+    """Algorithmic HBM bytes of one decode step at cache length L (before the step):
+    every weight once, K and V of L+1 keys per (sequence, KV head), the new K/V
+    written, and the activations in and out."""
+    es = 2
+    d, f, H, Hkv, dh, B = cfg.d, cfg.f, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.B
+    weights = ((H + 2 * Hkv) * dh * d + d * H * dh + 3 * d * f + 2 * d) * es
+    kv_read = 2 * B * Hkv * (L + 1) * dh * es
+    kv_write = 2 * B * Hkv * dh * es
+    act = 2 * B * d * es
+    return weights + kv_read + kv_write + act
+
+
+def decode_attn_bytes(cfg, L: int) -> int:
+    return 2 * cfg.B * cfg.n_kv_heads * (L + 1) * cfg.head_dim * 2
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        out = ROOT / "gpurun_out"
+        out.mkdir(exist_ok=True)
+        self.path = out / f"clocks_gpu{self.gpu}.csv"
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self) -> dict:
+        if not self.proc or not self.path or not self.path.exists():
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in self.path.read_text().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        load = [s for s, p in zip(sm, pw) if p is not None and p > 250] or sm
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def cpu_oracle_sample(cfg, W=None, X=None) -> dict:
+    """Time the fp64 oracle on the first CPU_SAMPLE_T tokens of the prefill
+    workload (a complete causal prefill of that length). Returns tokens/s."""
+    import numpy as np
+    from oracle import block as ob
+    from synth import make_weights, make_x
+
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count() or 1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    if W is None:
+        W = make_weights(cfg)
+    if X is None:
+        X = make_x(cfg)
+    Xs = X[:, :CPU_SAMPLE_T]
+    Wn = {k: np.asarray(v.to(dtype=__import__("torch").float64).numpy()) for k, v in W.items()}
+    t0 = time.perf_counter()
+    ob.block_prefill(Xs, Wn, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.eps, cfg.rope_base)
+    dt = time.perf_counter() - t0
+    return {"value": cfg.B * CPU_SAMPLE_T / dt, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, full prefill of the first {CPU_SAMPLE_T} tokens of the "
+                      f"7B-shaped block (B=1), {dt:.2f} s", "seconds": dt}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from synth import LLAMA7B, make_weights, make_x
+
+    cfg = LLAMA7B
+    W, X = make_weights(cfg), make_x(cfg)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(cfg, W, X)
+    samples = [cpu_oracle_sample(cfg, W, X) for _ in range(args.steps)]
+    secs = sum(s["seconds"] for s in samples)
+    value = cfg.B * CPU_SAMPLE_T * args.steps / secs
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"llama7b block prefill, first {CPU_SAMPLE_T} of T=2048 tokens per step "
+                               "(fp64 CPU oracle)", "d": cfg.d, "n_heads": cfg.n_heads, "head_dim": cfg.head_dim,
+                   "f": cfg.f, "B": cfg.B, "T": CPU_SAMPLE_T},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": samples[0]["cores"], "kind": "oracle",
+                         "sample": samples[0]["sample"].rsplit(",", 1)[0]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    import llama_pre_norm_b200 as lb
+    from synth import DECODE7B, LLAMA7B, make_weights, make_x
+
+    peaks = measured_peaks()
+    cfg = LLAMA7B
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    W = make_weights(cfg)
+    X = make_x(cfg)
+    Wd = {k: v.to(dev) for k, v in W.items()}
+    blk = lb.LlamaBlock(cfg.d, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.f, cfg.eps, cfg.rope_base,
+                        torch.bfloat16, max_pos=DECODE7B.cache_len + args.decode_steps + 64)
+    blk.set_weights(Wd)
+    blk.reserve(cfg.B * cfg.T, DECODE7B.B)
+    x = X.to(dev)
+    y = torch.empty_like(x)
+    kc = torch.zeros(cfg.B, cfg.n_kv_heads, cfg.T, cfg.head_dim, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    lens = torch.zeros(cfg.B, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------- prefill: warm-up, then K timed steps
+    for _ in range(args.warmup):
+        blk.prefill(x, y, kc, vc, lens)
+    blk.sync_status()
+    blk.enable_timing(True)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stage_ms: dict = {}
+    launches0 = blk.launch_count
+    clocks = ClockSampler(local)
+    with clocks:
+        barrier()
+        for i in range(args.steps):
+            flush.zero_()  # evict L2 outside the timed interval
+            starts[i].record(stream)
+            blk.prefill(x, y, kc, vc, lens)
+            ends[i].record(stream)
+            for name, ms in blk.stage_times():
+                stage_ms.setdefault(name, []).append(ms)
+        barrier()
+        prefill_launches = blk.launch_count - launches0
+        step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+        blk.sync_status()
+        tot_ms = max_over_ranks(sum(step_ms))
+
+        # ---------------- decode: B=32, cache 4096 -> 4096 + decode_steps
+        dec = None
+        if not args.no_decode:
+            dcfg = DECODE7B
+            t_max = dcfg.cache_len + args.decode_steps
+            g = torch.Generator(device=dev).manual_seed(2)
+            kcd = torch.zeros(dcfg.B, dcfg.n_kv_heads, t_max, dcfg.head_dim, dtype=torch.bfloat16, device=dev)
+            vcd = torch.zeros_like(kcd)
+            kcd[:, :, :dcfg.cache_len].normal_(generator=g)
+            vcd[:, :, :dcfg.cache_len].normal_(generator=g)
+            xs = torch.randn(args.decode_steps, dcfg.B, 1, dcfg.d, generator=g, device=dev).to(torch.bfloat16)
+            yd = torch.empty(dcfg.B, 1, dcfg.d, dtype=torch.bfloat16, device=dev)
+            dlens = torch.full((dcfg.B,), dcfg.cache_len, dtype=torch.int32, device=dev)
+
+            def reset():
+                dlens.fill_(dcfg.cache_len)
+                blk.set_lengths([dcfg.cache_len] * dcfg.B)
+
+            blk.enable_timing(False)
+            reset()
+            for s in range(min(args.warmup, args.decode_steps)):
+                blk.decode(xs[s], yd, kcd, vcd, dlens)
+            blk.sync_status()
+            reps = 2
+            dec_ms, attn_ms = [], []
+            dl0 = blk.launch_count
+            barrier()
+            for r in range(reps):
+                reset()
+                blk.enable_timing(r == reps - 1)  # stage timing on the last repetition
+                ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                ev0.record(stream)
+                for s in range(args.decode_steps):
+                    blk.decode(xs[s], yd, kcd, vcd, dlens)
+                    if r == reps - 1:
+                        for name, ms in blk.stage_times():
+                            if name == "attention":
+                                attn_ms.append(ms)
+                ev1.record(stream)
+                ev1.synchronize()
+                dec_ms.append(ev0.elapsed_time(ev1))
+            barrier()
+            blk.sync_status()
+            dec_launches = blk.launch_count - dl0
+            blk.enable_timing(False)
+            # the untimed-stage repetition is the headline (no events between kernels)
+            per_step_ms = max_over_ranks(dec_ms[0]) / args.decode_steps
+            Ls = range(dcfg.cache_len, dcfg.cache_len + args.decode_steps)
+            bytes_mean = statistics.mean(decode_bytes(dcfg, L) for L in Ls)
+            attn_bytes_mean = statistics.mean(decode_attn_bytes(dcfg, L) for L in Ls)
+            gbs = bytes_mean / (per_step_ms * 1e-3) / 1e9
+            attn_gbs = attn_bytes_mean / (statistics.mean(attn_ms) * 1e-3) / 1e9
+            dec = {
+                "workload": f"llama7b decode B={dcfg.B}, cache {dcfg.cache_len} -> {dcfg.cache_len + args.decode_steps}",
+                "ms_per_step": per_step_ms, "hbm_gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                "bytes_per_step_mean": bytes_mean, "tokens_per_s": dcfg.B / (per_step_ms * 1e-3) * world,
+                "steps": args.decode_steps, "repetitions": reps, "kernel_launches": dec_launches,
+                "attention_kernel": {"ms": statistics.mean(attn_ms), "bytes_mean": attn_bytes_mean,
+                                     "achieved_gbs": attn_gbs, "frac": attn_gbs / peaks["hbm_gbs"],
+                                     "traffic": NCU_TRAFFIC_BYTES["attention_decode"]},
+            }
+    clk = clocks.summary()
+
+    # ---------------- e2e: host buffers, copies inside the timed region
+    xh = X.pin_memory()
+    yh = torch.empty(X.shape, dtype=torch.bfloat16).pin_memory()
+    xe = torch.empty_like(x)
+    e2e_ms = []
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        xe.copy_(xh, non_blocking=True)
+        blk.prefill(xe, y, kc, vc, lens)
+        yh.copy_(y, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+    barrier()
+    e2e_tot = max_over_ranks(sum(e2e_ms))
+    blk.sync_status()
+
+    tokens = cfg.B * cfg.T
+    flops = prefill_flops(cfg)
+    ms_per_step = tot_ms / args.steps
+    value = tokens * args.steps * world / (tot_ms * 1e-3)
+    gu_ms = statistics.mean(stage_ms["gate_up_swiglu_gemm"])
+    gu_tflops = flops["gate_up"] / (gu_ms * 1e-3) / 1e12
+    stages = {k: round(statistics.mean(v), 4) for k, v in stage_ms.items()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        c = cpu_oracle_sample(cfg, W, X)
+        cpu = {k: c[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,0.02) weights, N(0,1) input)",
+        "config": {"workload": "llama7b block prefill, bf16, d=4096, 32 heads x 128, f=11008, B=1, T=2048",
+                   "global_batch": cfg.B * world, "seq_len": cfg.T,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed before every timed step (256 MB write)"},
+        "prefill": {"tflops": flops["total"] / (ms_per_step * 1e-3) / 1e12,
+                    "frac_of_bf16_peak": flops["total"] / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                    "gflop_per_step": flops["total"] / 1e9, "stage_ms": stages},
+        "decode": dec,
+        "roofline": {"kernel": "gate_up_swiglu_gemm", "bound": "tensor", "achieved": gu_tflops,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": gu_tflops / peaks["bf16_tflops"],
+                     "traffic": NCU_TRAFFIC_BYTES["gate_up_swiglu_gemm"],
+                     "peak_source": f"{peaks['source']} bf16 burst (kernel timed alone within a short step)",
+                     "algorithmic_flop_per_launch": flops["gate_up"]},
+        "cpu_baseline": cpu,
+        "e2e": {"value": tokens * args.steps * world / (e2e_tot * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": X.numel() * 2},
+        "gpu_launches": prefill_launches + (dec["kernel_launches"] if dec else 0),
+        "clocks": clk,
+    }
+    blk.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

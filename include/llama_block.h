@@ -115,8 +115,9 @@ size_t llama_block_kv_cache_bytes(int B, int n_kv_heads, int head_dim, int t_max
 
 /* Synchronise `stream`, read and clear the device error word (of the handle, or
  * of the standalone entry points when blk is NULL). Returns LB_OK, LB_ERR_TIMEOUT
- * (a bounded wait ran out, or a device-side bounds guard fired; details in
- * last_error) or LB_ERR_CUDA. */
+ * (a bounded wait ran out), LB_ERR_CACHE_FULL (a device-side bounds guard fired:
+ * a cache index or RoPE position out of range; the write was skipped) or
+ * LB_ERR_CUDA; details in last_error. */
 lb_status llama_block_sync_status(llama_block* blk, void* stream);
 
 /* Free the handle and everything it owns (synchronises the device first). */
@@ -124,6 +125,22 @@ void llama_block_destroy(llama_block* blk);
 
 /* Thread-local description of the last error (never NULL). */
 const char* llama_block_last_error(void);
+
+/* Profiling aid: when enabled, prefill and decode bracket each of their stages
+ * (one or two kernel launches) with CUDA events recorded on the caller's stream.
+ * Off by default; events are created on first enable. */
+lb_status llama_block_enable_timing(llama_block* blk, int enable);
+
+/* Device durations (ms) of the stages of the last prefill/decode call with timing
+ * enabled; waits for that call's events. Writes up to max_stages values into ms
+ * (may be NULL) and the stage count into *n_stages. */
+lb_status llama_block_stage_times(llama_block* blk, float* ms, int max_stages, int* n_stages);
+
+/* Name of stage i of the last prefill/decode call ("" when out of range). */
+const char* llama_block_stage_name(const llama_block* blk, int i);
+
+/* Number of kernels this handle has launched since it was created. */
+unsigned long long llama_block_launch_count(const llama_block* blk);
 
 /* Self-test of the bounded-wait machinery: launch one kernel that waits on a
  * device barrier that nothing completes, with a budget of `budget_ns`
@@ -135,7 +152,8 @@ lb_status llama_block_selftest_timeout(long long budget_ns, void* stream);
 /* ---------------- standalone entry points (testing) ---------------- */
 
 /* RMSNorm (LMDrive page §2.1; mechanics page §02.3): y = g * x / sqrt(mean(x^2) + eps)
- * over the last axis, fp32 accumulation, one rounding. x, y: [rows, d]; g: [d]. */
+ * over the last axis, fp32 accumulation, one rounding. x, y: [rows, d]; g: [d].
+ * rows == 0 is a no-op (pointers may then be NULL). */
 lb_status rmsnorm(const void* x, const void* g, void* y, int rows, int d, float eps,
                   lb_dtype dtype, void* stream);
 

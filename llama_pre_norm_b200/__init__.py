@@ -21,7 +21,8 @@ __all__ = [
     "llama_block_create", "llama_block_set_weights", "llama_block_reserve",
     "llama_block_prefill", "llama_block_decode", "llama_block_set_lengths",
     "llama_block_kv_cache_bytes", "llama_block_sync_status", "llama_block_destroy",
-    "llama_block_last_error", "llama_block_selftest_timeout",
+    "llama_block_last_error", "llama_block_selftest_timeout", "llama_block_enable_timing",
+    "llama_block_stage_times", "llama_block_stage_name", "llama_block_launch_count",
     "rmsnorm", "rope_apply", "causal_attn", "swiglu_mlp", "LlamaBlock",
 ]
 
@@ -50,6 +51,10 @@ _SIGS = {
     "llama_block_destroy": (None, [_p]),
     "llama_block_last_error": (ctypes.c_char_p, []),
     "llama_block_selftest_timeout": (_i, [_ll, _p]),
+    "llama_block_enable_timing": (_i, [_p, _i]),
+    "llama_block_stage_times": (_i, [_p, _p, _i, ctypes.POINTER(ctypes.c_int)]),
+    "llama_block_stage_name": (ctypes.c_char_p, [_p, _i]),
+    "llama_block_launch_count": (ctypes.c_ulonglong, [_p]),
     "rmsnorm": (_i, [_p, _p, _p, _i, _i, _f, _i, _p]),
     "rope_apply": (_i, [_p, _p, _i, _i, _i, _i, _f, _i, _p]),
     "causal_attn": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p]),
@@ -167,6 +172,26 @@ def llama_block_selftest_timeout(budget_ns: int, stream=None):
     _check(lib.llama_block_selftest_timeout(int(budget_ns), _stream(stream)), "llama_block_selftest_timeout")
 
 
+def llama_block_enable_timing(h, enable=True):
+    _check(lib.llama_block_enable_timing(h, 1 if enable else 0), "llama_block_enable_timing")
+
+
+def llama_block_stage_times(h) -> list:
+    """[(stage name, device ms)] of the last prefill/decode call (timing enabled)."""
+    n = ctypes.c_int(0)
+    buf = (ctypes.c_float * 16)()
+    _check(lib.llama_block_stage_times(h, buf, 16, ctypes.byref(n)), "llama_block_stage_times")
+    return [(llama_block_stage_name(h, i), float(buf[i])) for i in range(n.value)]
+
+
+def llama_block_stage_name(h, i) -> str:
+    return lib.llama_block_stage_name(h, i).decode()
+
+
+def llama_block_launch_count(h) -> int:
+    return int(lib.llama_block_launch_count(h))
+
+
 # ----------------------------------------------------------------- standalone entry points
 def rmsnorm(x, g, y, eps, stream=None):
     d = x.shape[-1]
@@ -228,6 +253,16 @@ class LlamaBlock:
 
     def sync_status(self, stream=None):
         llama_block_sync_status(self.handle, stream)
+
+    def enable_timing(self, enable=True):
+        llama_block_enable_timing(self.handle, enable)
+
+    def stage_times(self) -> list:
+        return llama_block_stage_times(self.handle)
+
+    @property
+    def launch_count(self) -> int:
+        return llama_block_launch_count(self.handle)
 
     def close(self):
         if self.handle:

@@ -143,7 +143,26 @@ struct llama_block {
   void* ws = nullptr;
   size_t ws_bytes = 0;
   std::vector<int> lens;  // host mirror of the cache lengths
+  // profiling: optional per-stage events, and the number of kernels launched
+  bool timing = false;
+  std::vector<cudaEvent_t> ev;            // 2 per stage
+  std::vector<const char*> stage_names;   // stages of the last prefill/decode
+  unsigned long long launches = 0;
 };
+
+static constexpr int kMaxStages = 16;
+
+// Run one stage (one or more kernel launches) on stream s, bracketed by events
+// when timing is enabled, and count its kernels.
+#define LB_STAGE(name, nkern, call)                                                  \
+  do {                                                                               \
+    const int si_ = (int)b->stage_names.size();                                      \
+    if (b->timing && si_ < kMaxStages) LB_CUDA(cudaEventRecord(b->ev[2 * si_], s));   \
+    LB_CUDA(call);                                                                   \
+    if (b->timing && si_ < kMaxStages) LB_CUDA(cudaEventRecord(b->ev[2 * si_ + 1], s)); \
+    b->stage_names.push_back(name);                                                  \
+    b->launches += (nkern);                                                          \
+  } while (0)
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -329,6 +348,7 @@ lb_status llama_block_create(int d, int n_heads, int n_kv_heads, int head_dim, i
 void llama_block_destroy(llama_block* b) {
   if (!b) return;
   cudaDeviceSynchronize();
+  for (cudaEvent_t e : b->ev) cudaEventDestroy(e);
   for (void* p : {b->w_qkv, b->w_o, b->w_gu, b->w_d, b->g1, b->g2, (void*)b->cos_t,
                   (void*)b->sin_t, (void*)b->err, b->ws})
     if (p) cudaFree(p);
@@ -425,44 +445,52 @@ lb_status llama_block_prefill(llama_block* b, const void* x, void* y, int B, int
   PrefillWs w = carve_prefill(b, b->ws, M, &need);
   const int d = b->d, H = b->H, Hkv = b->Hkv, dh = b->dh, f = b->f;
 
+  b->stage_names.clear();
   if (b->dtype == kBF16) {
-    LB_CUDA(launch_resid_rmsnorm(kBF16, x, nullptr, 0, 0, nullptr, b->g1, w.h, M, d, b->eps, s));
+    LB_STAGE("rmsnorm_attn", 1,
+             launch_resid_rmsnorm(kBF16, x, nullptr, 0, 0, nullptr, b->g1, w.h, M, d, b->eps, s));
     GemmEpi e1;
     e1.kind = kEpiQkvRope;
     e1.T = T; e1.H = H; e1.Hkv = Hkv; e1.dh = dh; e1.t_max = t_max; e1.max_pos = b->max_pos;
     e1.q_out = w.q; e1.k_cache = k_cache; e1.v_cache = v_cache;
     e1.cos_t = b->cos_t; e1.sin_t = b->sin_t; e1.err = b->err;
-    LB_CUDA(launch_gemm_tc(w.h, b->w_qkv, M, b->n_qkv, d, 256, 1, e1, b->num_sms, s));
-    LB_CUDA(launch_attn_tc(w.q, k_cache, v_cache, w.o, B, T, T, H, Hkv, dh, t_max, b->err, s));
+    LB_STAGE("qkv_rope_gemm", 1, launch_gemm_tc(w.h, b->w_qkv, M, b->n_qkv, d, 256, 1, e1, b->num_sms, s));
+    LB_STAGE("attention", 1,
+             launch_attn_tc(w.q, k_cache, v_cache, w.o, B, T, T, H, Hkv, dh, t_max, b->err, s));
     GemmEpi e2;
     e2.kind = kEpiResid; e2.out = w.x1; e2.resid = x; e2.ldo = d; e2.err = b->err;
-    LB_CUDA(launch_gemm_tc(w.o, b->w_o, M, d, H * dh, 256, 1, e2, b->num_sms, s));
-    LB_CUDA(launch_resid_rmsnorm(kBF16, w.x1, nullptr, 0, 0, nullptr, b->g2, w.h, M, d, b->eps, s));
+    LB_STAGE("o_proj_resid_gemm", 1, launch_gemm_tc(w.o, b->w_o, M, d, H * dh, 256, 1, e2, b->num_sms, s));
+    LB_STAGE("rmsnorm_mlp", 1,
+             launch_resid_rmsnorm(kBF16, w.x1, nullptr, 0, 0, nullptr, b->g2, w.h, M, d, b->eps, s));
     GemmEpi e3;
     e3.kind = kEpiSwiGLU; e3.out = w.a; e3.ldo = f; e3.f = f; e3.err = b->err;
-    LB_CUDA(launch_gemm_tc(w.h, b->w_gu, M, b->n_gu, d, 256, 1, e3, b->num_sms, s));
+    LB_STAGE("gate_up_swiglu_gemm", 1, launch_gemm_tc(w.h, b->w_gu, M, b->n_gu, d, 256, 1, e3, b->num_sms, s));
     GemmEpi e4;
     e4.kind = kEpiResid; e4.out = y; e4.resid = w.x1; e4.ldo = d; e4.err = b->err;
-    LB_CUDA(launch_gemm_tc(w.a, b->w_d, M, d, f, 256, 1, e4, b->num_sms, s));
+    LB_STAGE("down_resid_gemm", 1, launch_gemm_tc(w.a, b->w_d, M, d, f, 256, 1, e4, b->num_sms, s));
   } else {
     const float* X = (const float*)x;
-    LB_CUDA(launch_resid_rmsnorm(kF32, x, nullptr, 0, 0, nullptr, b->g1, w.h, M, d, b->eps, s));
-    LB_CUDA(launch_gemm_f32((const float*)w.h, (const float*)b->w_qkv, w.qkv32, nullptr, M,
-                            b->n_qkv, d, s));
-    LB_CUDA(launch_qkv_finish(kF32, w.qkv32, 1, 0, M, T, H, Hkv, dh, nullptr, b->cos_t, b->sin_t,
-                              b->max_pos, w.q, k_cache, v_cache, t_max, b->err, s));
-    LB_CUDA(launch_attn_f32((const float*)w.q, (const float*)k_cache, (const float*)v_cache,
-                            (float*)w.o, B, T, T, H, Hkv, dh, t_max, nullptr, s));
-    LB_CUDA(launch_gemm_f32((const float*)w.o, (const float*)b->w_o, (float*)w.x1, X, M, d,
-                            H * dh, s));
-    LB_CUDA(launch_resid_rmsnorm(kF32, w.x1, nullptr, 0, 0, nullptr, b->g2, w.h, M, d, b->eps, s));
-    LB_CUDA(launch_gemm_f32((const float*)w.h, (const float*)b->w_gu, w.gu32, nullptr, M, b->n_gu,
-                            d, s));
-    LB_CUDA(launch_silu_mul(kF32, w.gu32, 1, 0, M, f, b->n_gu, 0, w.a, s));
-    LB_CUDA(launch_gemm_f32((const float*)w.a, (const float*)b->w_d, (float*)y,
-                            (const float*)w.x1, M, d, f, s));
+    LB_STAGE("rmsnorm_attn", 1,
+             launch_resid_rmsnorm(kF32, x, nullptr, 0, 0, nullptr, b->g1, w.h, M, d, b->eps, s));
+    LB_STAGE("qkv_gemm", 1, launch_gemm_f32((const float*)w.h, (const float*)b->w_qkv, w.qkv32, nullptr, M,
+                                            b->n_qkv, d, s));
+    LB_STAGE("qkv_rope", 1, launch_qkv_finish(kF32, w.qkv32, 1, 0, M, T, H, Hkv, dh, nullptr, b->cos_t,
+                                              b->sin_t, b->max_pos, w.q, k_cache, v_cache, t_max,
+                                              b->err, s));
+    LB_STAGE("attention", 1, launch_attn_f32((const float*)w.q, (const float*)k_cache,
+                                             (const float*)v_cache, (float*)w.o, B, T, T, H, Hkv, dh,
+                                             t_max, nullptr, s));
+    LB_STAGE("o_proj_resid_gemm", 1, launch_gemm_f32((const float*)w.o, (const float*)b->w_o,
+                                                     (float*)w.x1, X, M, d, H * dh, s));
+    LB_STAGE("rmsnorm_mlp", 1,
+             launch_resid_rmsnorm(kF32, w.x1, nullptr, 0, 0, nullptr, b->g2, w.h, M, d, b->eps, s));
+    LB_STAGE("gate_up_gemm", 1, launch_gemm_f32((const float*)w.h, (const float*)b->w_gu, w.gu32, nullptr,
+                                                M, b->n_gu, d, s));
+    LB_STAGE("silu_mul", 1, launch_silu_mul(kF32, w.gu32, 1, 0, M, f, b->n_gu, 0, w.a, s));
+    LB_STAGE("down_resid_gemm", 1, launch_gemm_f32((const float*)w.a, (const float*)b->w_d, (float*)y,
+                                                   (const float*)w.x1, M, d, f, s));
   }
-  LB_CUDA(launch_set_lens(cache_len, B, T, s));
+  LB_STAGE("set_lengths", 1, launch_set_lens(cache_len, B, T, s));
   b->lens.assign(B, T);
   return LB_OK;
 }
@@ -486,64 +514,100 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
   DecodeWs w = carve_decode(b, b->ws, B, t_max, &need);
   const int d = b->d, H = b->H, Hkv = b->Hkv, dh = b->dh, f = b->f;
 
+  b->stage_names.clear();
   if (b->dtype == kBF16) {
     const int bn = B <= 32 ? 32 : B <= 64 ? 64 : B <= 128 ? 128 : 256;
-    LB_CUDA(launch_resid_rmsnorm(kBF16, x, nullptr, 0, 0, nullptr, b->g1, w.h, B, d, b->eps, s));
+    LB_STAGE("rmsnorm_attn", 1,
+             launch_resid_rmsnorm(kBF16, x, nullptr, 0, 0, nullptr, b->g1, w.h, B, d, b->eps, s));
     // Q|K|V: part[s][token][feature]
     GemmEpi e;
     e.kind = kEpiPartialT; e.out = w.part; e.err = b->err;
     e.ldo = b->n_qkv; e.split_stride = (long long)B * b->n_qkv;
     const int s1 = decode_split((b->n_qkv + 127) / 128, d);
-    LB_CUDA(launch_gemm_tc(b->w_qkv, w.h, b->n_qkv, B, d, bn, s1, e, b->num_sms, s));
-    const int s1e = gemm_effective_split(d, s1);
-    LB_CUDA(launch_qkv_finish(kBF16, w.part, s1e, e.split_stride, B, 1, H, Hkv, dh, cache_len,
-                              b->cos_t, b->sin_t, b->max_pos, w.q, k_cache, v_cache, t_max, b->err,
-                              s));
-    LB_CUDA(launch_attn_decode(w.q, k_cache, v_cache, w.o, w.attn_part, B, H, Hkv, dh, t_max,
-                               cache_len, b->err, s));
+    LB_STAGE("qkv_gemm", 1, launch_gemm_tc(b->w_qkv, w.h, b->n_qkv, B, d, bn, s1, e, b->num_sms, s));
+    LB_STAGE("qkv_rope_append", 1,
+             launch_qkv_finish(kBF16, w.part, gemm_effective_split(d, s1), e.split_stride, B, 1, H,
+                               Hkv, dh, cache_len, b->cos_t, b->sin_t, b->max_pos, w.q, k_cache,
+                               v_cache, t_max, b->err, s));
+    LB_STAGE("attention", 2, launch_attn_decode(w.q, k_cache, v_cache, w.o, w.attn_part, B, H, Hkv,
+                                                dh, t_max, cache_len, b->err, s));
     // o_proj, then X' = X + sum(partials) and h2 = RMSNorm(X') in one kernel
     const int K2 = H * dh;
     const int s2 = decode_split((d + 127) / 128, K2);
     e.ldo = d; e.split_stride = (long long)B * d;
-    LB_CUDA(launch_gemm_tc(b->w_o, w.o, d, B, K2, bn, s2, e, b->num_sms, s));
-    const int s2e = gemm_effective_split(K2, s2);
-    LB_CUDA(launch_resid_rmsnorm(kBF16, x, w.part, s2e, e.split_stride, w.x1, b->g2, w.h, B, d,
-                                 b->eps, s));
+    LB_STAGE("o_proj_gemm", 1, launch_gemm_tc(b->w_o, w.o, d, B, K2, bn, s2, e, b->num_sms, s));
+    LB_STAGE("resid_rmsnorm_mlp", 1,
+             launch_resid_rmsnorm(kBF16, x, w.part, gemm_effective_split(K2, s2), e.split_stride,
+                                  w.x1, b->g2, w.h, B, d, b->eps, s));
     // gate/up (packed rows), SiLU(g) * u
     const int s3 = decode_split((b->n_gu + 127) / 128, d);
     e.ldo = b->n_gu; e.split_stride = (long long)B * b->n_gu;
-    LB_CUDA(launch_gemm_tc(b->w_gu, w.h, b->n_gu, B, d, bn, s3, e, b->num_sms, s));
-    const int s3e = gemm_effective_split(d, s3);
-    LB_CUDA(launch_silu_mul(kBF16, w.part, s3e, e.split_stride, B, f, b->n_gu, 128, w.a, s));
+    LB_STAGE("gate_up_gemm", 1, launch_gemm_tc(b->w_gu, w.h, b->n_gu, B, d, bn, s3, e, b->num_sms, s));
+    LB_STAGE("silu_mul", 1, launch_silu_mul(kBF16, w.part, gemm_effective_split(d, s3), e.split_stride,
+                                            B, f, b->n_gu, 128, w.a, s));
     // down, y = X' + sum(partials); cache_len += 1
     const int s4 = decode_split((d + 127) / 128, f);
     e.ldo = d; e.split_stride = (long long)B * d;
-    LB_CUDA(launch_gemm_tc(b->w_d, w.a, d, B, f, bn, s4, e, b->num_sms, s));
-    const int s4e = gemm_effective_split(f, s4);
-    LB_CUDA(launch_resid_add(kBF16, w.x1, w.part, s4e, e.split_stride, y, (long long)B * d,
-                             cache_len, B, 1, s));
+    LB_STAGE("down_gemm", 1, launch_gemm_tc(b->w_d, w.a, d, B, f, bn, s4, e, b->num_sms, s));
+    LB_STAGE("resid_add_len", 1, launch_resid_add(kBF16, w.x1, w.part, gemm_effective_split(f, s4),
+                                                  e.split_stride, y, (long long)B * d, cache_len, B,
+                                                  1, s));
   } else {
     const float* X = (const float*)x;
-    LB_CUDA(launch_resid_rmsnorm(kF32, x, nullptr, 0, 0, nullptr, b->g1, w.h, B, d, b->eps, s));
-    LB_CUDA(launch_gemm_f32((const float*)w.h, (const float*)b->w_qkv, w.part, nullptr, B,
-                            b->n_qkv, d, s));
-    LB_CUDA(launch_qkv_finish(kF32, w.part, 1, 0, B, 1, H, Hkv, dh, cache_len, b->cos_t, b->sin_t,
-                              b->max_pos, w.q, k_cache, v_cache, t_max, b->err, s));
-    LB_CUDA(launch_attn_f32((const float*)w.q, (const float*)k_cache, (const float*)v_cache,
-                            (float*)w.o, B, 1, 1, H, Hkv, dh, t_max, cache_len, s));
-    LB_CUDA(launch_gemm_f32((const float*)w.o, (const float*)b->w_o, (float*)w.x1, X, B, d,
-                            H * dh, s));
-    LB_CUDA(launch_resid_rmsnorm(kF32, w.x1, nullptr, 0, 0, nullptr, b->g2, w.h, B, d, b->eps, s));
-    LB_CUDA(launch_gemm_f32((const float*)w.h, (const float*)b->w_gu, w.part, nullptr, B, b->n_gu,
-                            d, s));
-    LB_CUDA(launch_silu_mul(kF32, w.part, 1, 0, B, f, b->n_gu, 0, w.a, s));
-    LB_CUDA(launch_gemm_f32((const float*)w.a, (const float*)b->w_d, (float*)y,
-                            (const float*)w.x1, B, d, f, s));
-    LB_CUDA(launch_resid_add(kF32, nullptr, nullptr, 0, 0, nullptr, 0, cache_len, B, 1, s));
+    LB_STAGE("rmsnorm_attn", 1,
+             launch_resid_rmsnorm(kF32, x, nullptr, 0, 0, nullptr, b->g1, w.h, B, d, b->eps, s));
+    LB_STAGE("qkv_gemm", 1, launch_gemm_f32((const float*)w.h, (const float*)b->w_qkv, w.part, nullptr,
+                                            B, b->n_qkv, d, s));
+    LB_STAGE("qkv_rope_append", 1,
+             launch_qkv_finish(kF32, w.part, 1, 0, B, 1, H, Hkv, dh, cache_len, b->cos_t, b->sin_t,
+                               b->max_pos, w.q, k_cache, v_cache, t_max, b->err, s));
+    LB_STAGE("attention", 1, launch_attn_f32((const float*)w.q, (const float*)k_cache,
+                                             (const float*)v_cache, (float*)w.o, B, 1, 1, H, Hkv, dh,
+                                             t_max, cache_len, s));
+    LB_STAGE("o_proj_resid_gemm", 1, launch_gemm_f32((const float*)w.o, (const float*)b->w_o,
+                                                     (float*)w.x1, X, B, d, H * dh, s));
+    LB_STAGE("rmsnorm_mlp", 1,
+             launch_resid_rmsnorm(kF32, w.x1, nullptr, 0, 0, nullptr, b->g2, w.h, B, d, b->eps, s));
+    LB_STAGE("gate_up_gemm", 1, launch_gemm_f32((const float*)w.h, (const float*)b->w_gu, w.part,
+                                                nullptr, B, b->n_gu, d, s));
+    LB_STAGE("silu_mul", 1, launch_silu_mul(kF32, w.part, 1, 0, B, f, b->n_gu, 0, w.a, s));
+    LB_STAGE("down_resid_gemm", 1, launch_gemm_f32((const float*)w.a, (const float*)b->w_d, (float*)y,
+                                                   (const float*)w.x1, B, d, f, s));
+    LB_STAGE("increment_lengths", 1,
+             launch_resid_add(kF32, nullptr, nullptr, 0, 0, nullptr, 0, cache_len, B, 1, s));
   }
   for (int i = 0; i < B; ++i) b->lens[i] += 1;
   return LB_OK;
 }
+
+lb_status llama_block_enable_timing(llama_block* b, int enable) {
+  if (!b) return fail(LB_ERR_INVALID_ARG, "enable_timing: NULL handle");
+  if (enable && b->ev.empty()) {
+    b->ev.resize(2 * kMaxStages);
+    for (auto& e : b->ev) LB_CUDA(cudaEventCreate(&e));
+  }
+  b->timing = enable != 0;
+  return LB_OK;
+}
+
+lb_status llama_block_stage_times(llama_block* b, float* ms, int max_stages, int* n_stages) {
+  if (!b || !n_stages) return fail(LB_ERR_INVALID_ARG, "stage_times: NULL argument");
+  if (!b->timing) return fail(LB_ERR_INVALID_ARG, "stage_times: timing is not enabled");
+  const int n = std::min((int)b->stage_names.size(), kMaxStages);
+  *n_stages = n;
+  for (int i = 0; i < n && i < max_stages && ms; ++i) {
+    LB_CUDA(cudaEventSynchronize(b->ev[2 * i + 1]));
+    LB_CUDA(cudaEventElapsedTime(&ms[i], b->ev[2 * i], b->ev[2 * i + 1]));
+  }
+  return LB_OK;
+}
+
+const char* llama_block_stage_name(const llama_block* b, int i) {
+  if (!b || i < 0 || i >= (int)b->stage_names.size()) return "";
+  return b->stage_names[i];
+}
+
+unsigned long long llama_block_launch_count(const llama_block* b) { return b ? b->launches : 0; }
 
 static const char* describe_err(int code) {
   if (code >= kErrWaitBase && code < kErrWaitBase + 0x100) return "a bounded device wait ran out";
@@ -581,8 +645,9 @@ static lb_status check_dtype(lb_dtype dt, const char* who) {
 lb_status rmsnorm(const void* x, const void* g, void* y, int rows, int d, float eps,
                   lb_dtype dtype, void* stream) {
   if (check_dtype(dtype, "rmsnorm") != LB_OK) return LB_ERR_INVALID_ARG;
-  if (!x || !g || !y) return fail(LB_ERR_INVALID_ARG, "rmsnorm: NULL pointer");
   if (rows < 0 || d <= 0 || !(eps > 0.f)) return fail(LB_ERR_INVALID_ARG, "rmsnorm: bad size");
+  if (rows == 0) return LB_OK;  // nothing to do; empty tensors may carry NULL pointers
+  if (!x || !g || !y) return fail(LB_ERR_INVALID_ARG, "rmsnorm: NULL pointer");
   if (d % 8 != 0 || d > 8192)
     return fail(LB_ERR_UNSUPPORTED, "rmsnorm: d must be a multiple of 8 and <= 8192");
   LB_CUDA(launch_resid_rmsnorm(dtype, x, nullptr, 0, 0, nullptr, g, y, rows, d, eps,

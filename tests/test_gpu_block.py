@@ -13,14 +13,13 @@ import torch
 
 from oracle import block as ob
 from synth import BlockConfig, TINY_F32, make_cache, make_decode_x, make_weights, make_x
-from tests.helpers import BF16_TOL, F32_TOL, as_np, cuda, rel_err_floor, row_err, weights_to_cuda
+from tests.helpers import BF16_TOL, F32_TOL, as_np, branch_err, cuda, row_err, weights_to_cuda
 
 pytestmark = pytest.mark.gpu
 
 if torch.cuda.is_available():
     import llama_pre_norm_b200 as lb
 
-BRANCH_TOL_BF16 = 5e-2  # X'' - X carries the bf16 rounding of X'' (|X| ~ 4 in a row)
 
 SMALL_BF16 = [
     BlockConfig("bf16-gqa", d=512, n_heads=4, n_kv_heads=2, head_dim=128, f=1408, B=2, T=200,
@@ -50,12 +49,12 @@ def _run_prefill(cfg, X, W, t_max):
     return blk, y, kc, vc, lens
 
 
-def _check(cfg, got, want, tol_rows=None):
-    if cfg.dtype == "f32":
-        assert rel_err_floor(got, want) <= F32_TOL
-        assert row_err(got, want) <= F32_TOL
-    else:
-        assert row_err(got, want) <= (tol_rows or BF16_TOL)
+def _tol(cfg):
+    return F32_TOL if cfg.dtype == "f32" else BF16_TOL
+
+
+def _check(cfg, got, want):
+    assert row_err(got, want) <= _tol(cfg)
 
 
 @pytest.mark.parametrize("cfg", [TINY_F32] + SMALL_BF16, ids=lambda c: c.name)
@@ -68,12 +67,8 @@ def test_block_prefill(cfg):
     _check(cfg, y, ref["y"])
     _check(cfg, kc[:, :, :cfg.T], ref["k"])
     _check(cfg, vc[:, :, :cfg.T], ref["v"])
-    branch = as_np(y) - as_np(X)
-    want_branch = ref["attn"] + ref["mlp"]
-    if cfg.dtype == "f32":
-        assert row_err(branch, want_branch) <= 10 * F32_TOL
-    else:
-        assert row_err(branch, want_branch) <= BRANCH_TOL_BF16
+    u = 2.0 ** -24 if cfg.dtype == "f32" else 2.0 ** -8
+    assert branch_err(y, ref["y"], ref["x1"], ref["attn"] + ref["mlp"], u) <= _tol(cfg)
     assert lens.tolist() == [cfg.T] * cfg.B
     blk.close()
 

@@ -42,7 +42,7 @@ CPU_SAMPLE_T = 2048  # tokens of the 7B prefill the CPU oracle evaluates per sam
 # DRAM traffic per launch of the dominant kernels from ncu captures (see
 # profiles/); None until a capture of the current kernel exists.
 NCU_TRAFFIC_BYTES = {
-    "gate_up_swiglu_gemm": None,
+    "gate_up_swiglu_gemm": 232_250_624,  # profiles/gemm_tc_gate_up_llama7b.md
     "attention_decode": None,
 }
 
@@ -98,6 +98,25 @@ def decode_bytes(cfg, L: int) -> int:
 
 def decode_attn_bytes(cfg, L: int) -> int:
     return 2 * cfg.B * cfg.n_kv_heads * (L + 1) * cfg.head_dim * 2
+
+
+# ------------------------------------------------------------------ replicas
+def reduce_max(v: float, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(units_per_rank_step: int, steps: int, world: int, slowest_ms: float) -> float:
+    """Whole-job throughput of independent replicas: every rank processes the same
+    units per step; the job takes as long as its slowest rank."""
+    return units_per_rank_step * steps * world / (slowest_ms * 1e-3)
 
 
 # ------------------------------------------------------------------ clocks
@@ -259,11 +278,7 @@ def run_ours(args):
         torch.cuda.synchronize()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, dev)
 
     # ---------------- prefill: warm-up, then K timed steps
     for _ in range(args.warmup):
@@ -376,7 +391,7 @@ def run_ours(args):
     tokens = cfg.B * cfg.T
     flops = prefill_flops(cfg)
     ms_per_step = tot_ms / args.steps
-    value = tokens * args.steps * world / (tot_ms * 1e-3)
+    value = replica_throughput(tokens, args.steps, world, tot_ms)
     gu_ms = statistics.mean(stage_ms["gate_up_swiglu_gemm"])
     gu_tflops = flops["gate_up"] / (gu_ms * 1e-3) / 1e12
     stages = {k: round(statistics.mean(v), 4) for k, v in stage_ms.items()}
@@ -404,7 +419,7 @@ def run_ours(args):
                      "peak_source": f"{peaks['source']} bf16 burst (kernel timed alone within a short step)",
                      "algorithmic_flop_per_launch": flops["gate_up"]},
         "cpu_baseline": cpu,
-        "e2e": {"value": tokens * args.steps * world / (e2e_tot * 1e-3), "unit": UNIT,
+        "e2e": {"value": replica_throughput(tokens, args.steps, world, e2e_tot), "unit": UNIT,
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": X.numel() * 2},
         "gpu_launches": prefill_launches + (dec["kernel_launches"] if dec else 0),
         "clocks": clk,

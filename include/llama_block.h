@@ -180,6 +180,33 @@ lb_status swiglu_mlp(const void* h, const void* w_gate, const void* w_up,
                      const void* w_down, void* y, int M, int d, int f, lb_dtype dtype,
                      void* stream);
 
+/* Decode attention that allocates nothing, for callers that may not call
+ * cudaMalloc (or any allocator) while they run: code inside a region whose
+ * device memory is budgeted up front, a host that hands all device memory to its
+ * own pool, or a launch path that must not synchronise the device the way an
+ * allocation or free can. The pages have no counterpart; it is an operational
+ * variant of the split-KV decode attention that llama_block_decode runs.
+ *
+ * Computes, for each sequence b and query head h, the attention of the single
+ * query q[b][h] (at position kv_len[b]) over keys 0..kv_len[b]:
+ *   q: [B, n_heads, head_dim]; k, v: [B, n_kv_heads, k_stride_T, head_dim];
+ *   kv_len: device int32 [B], kv_len[b] + 1 <= k_stride_T;
+ *   o: [B, n_heads * head_dim]; all bf16 except kv_len. The caller passes inputs
+ *   and outputs; the split-KV partials go to a fixed array inside the library.
+ * Limit: B * n_heads * ceil(k_stride_T / 128) * (head_dim + 2) <= 6 * 2^20 floats
+ * (24 MiB); larger calls return LB_ERR_INVALID_ARG before anything is launched.
+ * Every GPU that loads the library holds that array until the process exits.
+ * The first call on a device looks up the array's device address on that
+ * device; make that first call before any stream capture. All calls on one
+ * device share its array and it keeps the last call's contents, so calls that
+ * may overlap on that GPU (several streams, threads or processes) race:
+ * serialise them.
+ * A bounded wait that runs out ends the kernel early and sets a device word
+ * private to this entry point; the output of that call is then undefined. */
+lb_status decode_attn_static_scratch(const void* q, const void* k, const void* v, void* o,
+                                     const int32_t* kv_len, int B, int n_heads, int n_kv_heads,
+                                     int head_dim, int k_stride_T, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,7 +23,7 @@ __all__ = [
     "llama_block_kv_cache_bytes", "llama_block_sync_status", "llama_block_destroy",
     "llama_block_last_error", "llama_block_selftest_timeout", "llama_block_enable_timing",
     "llama_block_stage_times", "llama_block_stage_name", "llama_block_launch_count",
-    "rmsnorm", "rope_apply", "causal_attn", "swiglu_mlp", "LlamaBlock",
+    "rmsnorm", "rope_apply", "causal_attn", "swiglu_mlp", "decode_attn_static_scratch", "LlamaBlock",
 ]
 
 LB_F32, LB_BF16 = 0, 1
@@ -59,6 +59,7 @@ _SIGS = {
     "rope_apply": (_i, [_p, _p, _i, _i, _i, _i, _f, _i, _p]),
     "causal_attn": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p]),
     "swiglu_mlp": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _p]),
+    "decode_attn_static_scratch": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -222,6 +223,18 @@ def swiglu_mlp(h, w_gate, w_up, w_down, y, stream=None):
     _check(lib.swiglu_mlp(_ptr(h, "h"), _ptr(w_gate, "w_gate", h.dtype), _ptr(w_up, "w_up", h.dtype),
                           _ptr(w_down, "w_down", h.dtype), _ptr(y, "y", h.dtype), M, d, f,
                           dtype_code(h.dtype), _stream(stream)), "swiglu_mlp")
+
+
+def decode_attn_static_scratch(q, k, v, o, kv_len, stream=None):
+    """Decode attention that allocates no device memory (see the C header).
+    q [B, H, head_dim]; k, v [B, H_kv, k_stride, head_dim]; o [B, H * head_dim];
+    kv_len int32 [B] (query b sits at position kv_len[b] and sees keys 0..kv_len[b])."""
+    B, H, dh = q.shape
+    Hkv, ks = k.shape[1], k.shape[2]
+    _check(lib.decode_attn_static_scratch(_ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                          _ptr(v, "v", torch.bfloat16), _ptr(o, "o", torch.bfloat16),
+                                          _ptr(kv_len, "kv_len", torch.int32), B, H, Hkv, dh, ks,
+                                          _stream(stream)), "decode_attn_static_scratch")
 
 
 class LlamaBlock:

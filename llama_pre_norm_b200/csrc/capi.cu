@@ -748,3 +748,61 @@ lb_status swiglu_mlp(const void* h, const void* w_gate, const void* w_up, const 
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ static-scratch decode attention
+// For callers that may not allocate device memory, decode attention with its
+// split-KV partials kept in a fixed array of this file instead of a caller- or
+// library-allocated workspace. The array (kNoAllocScratchFloats floats, 24 MiB)
+// is part of the library image: every GPU that loads the library holds it until
+// the process exits. Its device address is looked up once per device.
+static constexpr size_t kNoAllocScratchFloats = (size_t)6 << 20;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+static __device__ int g_noalloc_err;
+
+struct NoAllocSlot {
+  float* scratch = nullptr;
+  int* err = nullptr;
+};
+static std::mutex g_noalloc_mu;
+static std::map<int, NoAllocSlot> g_noalloc_slots;
+
+extern "C" lb_status decode_attn_static_scratch(const void* q, const void* k, const void* v,
+                                                void* o, const int32_t* kv_len, int B,
+                                                int n_heads, int n_kv_heads, int head_dim,
+                                                int k_stride_T, void* stream) {
+  if (!q || !k || !v || !o || !kv_len)
+    return fail(LB_ERR_INVALID_ARG, "decode_attn_static_scratch: NULL pointer");
+  if (B <= 0 || n_heads <= 0 || n_kv_heads <= 0 || k_stride_T <= 0)
+    return fail(LB_ERR_INVALID_ARG, "decode_attn_static_scratch: sizes must be positive");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(LB_ERR_UNSUPPORTED, "decode_attn_static_scratch: head_dim %d not in {64,128}", head_dim);
+  if (n_heads % n_kv_heads || n_heads / n_kv_heads > 8)
+    return fail(LB_ERR_UNSUPPORTED, "decode_attn_static_scratch: need n_heads %% n_kv_heads == 0 "
+                                    "and at most 8 query heads per KV head");
+  const size_t need = (size_t)B * n_heads * decode_attn_chunks(k_stride_T) * (head_dim + 2);
+  if (need > kNoAllocScratchFloats)
+    return fail(LB_ERR_INVALID_ARG,
+                "decode_attn_static_scratch: B*n_heads*ceil(k_stride_T/128)*(head_dim+2) = %zu "
+                "floats exceeds the fixed scratch of %zu floats",
+                need, kNoAllocScratchFloats);
+  int dev = 0;
+  LB_CUDA(cudaGetDevice(&dev));
+  NoAllocSlot slot;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    auto it = g_noalloc_slots.find(dev);
+    if (it == g_noalloc_slots.end()) {
+      // first call on this device: resolve the device addresses of the arrays
+      LB_CUDA(cudaGetSymbolAddress((void**)&slot.scratch, g_noalloc_scratch));
+      LB_CUDA(cudaGetSymbolAddress((void**)&slot.err, g_noalloc_err));
+      g_noalloc_slots[dev] = slot;
+    } else {
+      slot = it->second;
+    }
+  }
+  // The partials need no clearing: every (sequence, head, chunk) slot the combine
+  // step reads is written by this call's split kernel first.
+  LB_CUDA(launch_attn_decode(q, k, v, o, slot.scratch, B, n_heads, n_kv_heads, head_dim, k_stride_T,
+                             kv_len, slot.err, (cudaStream_t)stream));
+  return LB_OK;
+}

@@ -26,7 +26,7 @@ def declared_functions():
 
 def test_library_exports_every_declared_function():
     names = declared_functions()
-    assert "llama_block_create" in names and "causal_attn" in names and len(names) == 19
+    assert "llama_block_create" in names and "causal_attn" in names and len(names) == 20
     for n in names:
         assert hasattr(lb.lib, n), f"{n} declared in llama_block.h but not exported"
 

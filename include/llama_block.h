@@ -26,7 +26,7 @@
  *    reason is available from llama_block_last_error() (thread-local string).
  *  - Device-side waits are bounded: a wait that runs out latches an error word on
  *    the device instead of hanging; llama_block_sync_status() reads it.
- *  - Restrictions: head_dim in {64, 128}; n_heads % n_kv_heads == 0;
+ *  - Restrictions: head_dim in {64, 128}; n_heads / n_kv_heads in {1, 2, 4, 8};
  *    n_heads * head_dim and d are multiples of 64 for LB_BF16; y must not alias x.
  *  - A handle is not thread-safe: do not call it concurrently from several threads.
  */
@@ -61,7 +61,8 @@ typedef struct llama_block llama_block; /* opaque, library-owned */
  * the library builds in fp64 on the host. Allocates library-owned device memory
  * (packed weights, RoPE table, error word) on the current device.
  * Returns LB_ERR_INVALID_ARG for non-positive sizes or a null `out`,
- * LB_ERR_UNSUPPORTED for head_dim not in {64,128} or n_heads % n_kv_heads != 0. */
+ * LB_ERR_UNSUPPORTED for head_dim not in {64,128} or n_heads / n_kv_heads not in
+ * {1, 2, 4, 8}. */
 lb_status llama_block_create(int d, int n_heads, int n_kv_heads, int head_dim, int f,
                              float eps, float rope_base, lb_dtype dtype, int max_pos,
                              llama_block** out);
@@ -193,7 +194,7 @@ lb_status swiglu_mlp(const void* h, const void* w_gate, const void* w_up,
  *   kv_len: device int32 [B], kv_len[b] + 1 <= k_stride_T;
  *   o: [B, n_heads * head_dim]; all bf16 except kv_len. The caller passes inputs
  *   and outputs; the split-KV partials go to a fixed array inside the library.
- * Limit: B * n_heads * ceil(k_stride_T / 128) * (head_dim + 2) <= 6 * 2^20 floats
+ * Limit: B * n_heads * ceil(k_stride_T / 512) * (head_dim + 2) <= 6 * 2^20 floats
  * (24 MiB); larger calls return LB_ERR_INVALID_ARG before anything is launched.
  * Every GPU that loads the library holds that array until the process exits.
  * The first call on a device looks up the array's device address on that

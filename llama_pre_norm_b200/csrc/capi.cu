@@ -275,8 +275,11 @@ lb_status llama_block_create(int d, int n_heads, int n_kv_heads, int head_dim, i
     return fail(LB_ERR_UNSUPPORTED, "create: head_dim %d not in {64,128}", head_dim);
   if (n_heads % n_kv_heads != 0)
     return fail(LB_ERR_UNSUPPORTED, "create: n_heads %% n_kv_heads != 0");
-  if (n_heads / n_kv_heads > 8)
-    return fail(LB_ERR_UNSUPPORTED, "create: more than 8 query heads per KV head");
+  {
+    const int rep = n_heads / n_kv_heads;
+    if (rep != 1 && rep != 2 && rep != 4 && rep != 8)
+      return fail(LB_ERR_UNSUPPORTED, "create: query heads per KV head must be 1, 2, 4 or 8");
+  }
   if (d % 8 != 0 || d > 8192)
     return fail(LB_ERR_UNSUPPORTED, "create: d must be a multiple of 8 and <= 8192");
   if (dtype == LB_BF16 && (d % 64 != 0 || f % 8 != 0 || (n_heads * head_dim) % 64 != 0))
@@ -776,13 +779,15 @@ extern "C" lb_status decode_attn_static_scratch(const void* q, const void* k, co
     return fail(LB_ERR_INVALID_ARG, "decode_attn_static_scratch: sizes must be positive");
   if (head_dim != 64 && head_dim != 128)
     return fail(LB_ERR_UNSUPPORTED, "decode_attn_static_scratch: head_dim %d not in {64,128}", head_dim);
-  if (n_heads % n_kv_heads || n_heads / n_kv_heads > 8)
-    return fail(LB_ERR_UNSUPPORTED, "decode_attn_static_scratch: need n_heads %% n_kv_heads == 0 "
-                                    "and at most 8 query heads per KV head");
+  if (n_heads % n_kv_heads ||
+      (n_heads / n_kv_heads != 1 && n_heads / n_kv_heads != 2 && n_heads / n_kv_heads != 4 &&
+       n_heads / n_kv_heads != 8))
+    return fail(LB_ERR_UNSUPPORTED, "decode_attn_static_scratch: query heads per KV head must be "
+                                    "1, 2, 4 or 8");
   const size_t need = (size_t)B * n_heads * decode_attn_chunks(k_stride_T) * (head_dim + 2);
   if (need > kNoAllocScratchFloats)
     return fail(LB_ERR_INVALID_ARG,
-                "decode_attn_static_scratch: B*n_heads*ceil(k_stride_T/128)*(head_dim+2) = %zu "
+                "decode_attn_static_scratch: B*n_heads*ceil(k_stride_T/512)*(head_dim+2) = %zu "
                 "floats exceeds the fixed scratch of %zu floats",
                 need, kNoAllocScratchFloats);
   int dev = 0;

@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(kDecThreads, NREP >= 4 ? 1 : 2) attn_decode_sp
   float* qs = reinterpret_cast<float*>(smem + kDecStages * 2 * CHUNK_BYTES);  // [NREP][DH]
   __shared__ __align__(8) uint64_t full[kDecStages], empty[kDecStages];
 
+  pdl_wait();
+  pdl_trigger();
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int nkeys = kv_len[b] + 1;  // cached keys plus the one just appended
   const int k0 = split * kDecSplitKeys;
@@ -254,6 +256,8 @@ __global__ void __launch_bounds__(kDecThreads, NREP >= 4 ? 1 : 2) attn_decode_sp
 template <int DH>
 __global__ void attn_decode_combine_kernel(const float* __restrict__ part, bf16* __restrict__ o,
                                            int H, int n_splits, const int* __restrict__ kv_len) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const int used = min(n_splits, (kv_len[b] + 1 + kDecSplitKeys - 1) / kDecSplitKeys);
   const float* base = part + ((long long)b * H + h) * n_splits * (DH + 2);
@@ -281,9 +285,8 @@ static cudaError_t run_split(dim3 grid, const void* q, const void* k, const void
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<grid, kDecThreads, smem, s>>>((const bf16*)q, (const bf16*)k, (const bf16*)v, part, H, Hkv,
-                                       k_stride, n_splits, kv_len, scale_log2, err);
-  return cudaGetLastError();
+  return launch_k(kern, grid, kDecThreads, smem, s, (const bf16*)q, (const bf16*)k, (const bf16*)v,
+                  part, H, Hkv, k_stride, n_splits, kv_len, scale_log2, err);
 }
 
 template <int DH>
@@ -302,8 +305,8 @@ static cudaError_t run_decode(const void* q, const void* k, const void* v, void*
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
-  attn_decode_combine_kernel<DH><<<dim3(H, B), DH, 0, s>>>(part, (bf16*)o, H, n_splits, kv_len);
-  return cudaGetLastError();
+  return launch_k(attn_decode_combine_kernel<DH>, dim3(H, B), DH, 0, s, (const float*)part,
+                  (bf16*)o, H, n_splits, kv_len);
 }
 
 cudaError_t launch_attn_decode(const void* q, const void* k, const void* v, void* o, float* part,

@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -116,6 +117,7 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
                       j * C::BKV, b * Hkv + hk);
         issued = j + 1;
       }
+      pdl_trigger();
       // every issued load must land before the CTA may exit
       mbar_wait(q_full, 0, err, 0x22);
       for (int j = max(0, issued - 2); j < issued; ++j) {
@@ -300,9 +302,8 @@ static cudaError_t run_attn(const void* q, const void* k, const void* v, void* o
   }
   const int nq = (Tq + 127) / 128;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
-  kern<<<nq * B * H, kAttnTcThreads, C::SMEM, s>>>(tq, tk, tv, (bf16*)o, B, Tq, Tk, H, Hkv,
-                                                   scale_log2, err);
-  return cudaGetLastError();
+  return launch_k(kern, nq * B * H, kAttnTcThreads, C::SMEM, s, tq, tk, tv, (bf16*)o, B, Tq, Tk, H,
+                  Hkv, scale_log2, err);
 }
 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, int B, int Tq,

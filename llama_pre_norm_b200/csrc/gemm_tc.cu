@@ -260,6 +260,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // inputs of the previous kernel are complete and visible from here on
 
   const int num_m = (M + kBM - 1) / kBM, num_n = (N + BN - 1) / BN;
   const int KB = (K + kBK - 1) / kBK;
@@ -288,6 +289,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+      pdl_trigger();  // all loads issued: the next kernel may start launching
       // Every load issued must land before the CTA may exit.
       const long long first = issued > C::STAGES ? issued - C::STAGES : 0;
       for (long long i = first; i < issued; ++i)
@@ -382,8 +384,7 @@ static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int M, int 
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<grid, kGemmThreads, C::SMEM, s>>>(ta, tb, M, N, K, kb_per, n_split, epi);
-  return cudaGetLastError();
+  return launch_k(kern, grid, kGemmThreads, C::SMEM, s, ta, tb, M, N, K, kb_per, n_split, epi);
 }
 
 cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, int BN, int n_split,

@@ -28,6 +28,27 @@ inline int gemm_effective_split(int K, int n_split) {
   return (KB + per - 1) / per;
 }
 
+// Launch `kern` on `s` with programmatic dependent launch allowed: the grid may
+// start while the previous kernel on the stream finishes. Every kernel of this
+// library executes griddepcontrol.wait (pdl_wait) before its first global-memory
+// access, so only its prologue (barrier init, TMEM allocation, descriptor
+// prefetch) overlaps the previous kernel.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ----------------------------------------------------------- norm_fuse.cu
 cudaError_t launch_resid_rmsnorm(int dtype, const void* x, const float* partial, int n_split,
                                  long long split_stride, void* x_out, const void* g, void* y,

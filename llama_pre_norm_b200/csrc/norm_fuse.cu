@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(kNormThreads) resid_rmsnorm_kernel(
     const T* __restrict__ x, const float* __restrict__ partial, int n_split, long long split_stride,
     T* __restrict__ x_out, const T* __restrict__ g, T* __restrict__ y, int d, float eps) {
   __shared__ float red[32];
+  pdl_wait();
+  pdl_trigger();
   const long long row = blockIdx.x;
   const int nvec = d >> 3;
   float v[kMaxVec][8];
@@ -72,14 +74,10 @@ cudaError_t launch_resid_rmsnorm(int dtype, const void* x, const float* partial,
                                  int rows, int d, float eps, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   if (dtype == kF32)
-    resid_rmsnorm_kernel<float><<<rows, kNormThreads, 0, s>>>(
-        (const float*)x, partial, n_split, split_stride, (float*)x_out, (const float*)g,
-        (float*)y, d, eps);
-  else
-    resid_rmsnorm_kernel<bf16><<<rows, kNormThreads, 0, s>>>(
-        (const bf16*)x, partial, n_split, split_stride, (bf16*)x_out, (const bf16*)g, (bf16*)y,
-        d, eps);
-  return cudaGetLastError();
+    return launch_k(resid_rmsnorm_kernel<float>, rows, kNormThreads, 0, s, (const float*)x, partial,
+                    n_split, split_stride, (float*)x_out, (const float*)g, (float*)y, d, eps);
+  return launch_k(resid_rmsnorm_kernel<bf16>, rows, kNormThreads, 0, s, (const bf16*)x, partial,
+                  n_split, split_stride, (bf16*)x_out, (const bf16*)g, (bf16*)y, d, eps);
 }
 
 // ---------------------------------------------------------------- QKV finish
@@ -97,6 +95,8 @@ __global__ void qkv_finish_kernel(const float* __restrict__ qkv, int n_split,
                                   const float* __restrict__ sin_t, int max_pos, T* __restrict__ q_out,
                                   T* __restrict__ k_cache, T* __restrict__ v_cache, int t_max,
                                   int* err) {
+  pdl_wait();
+  pdl_trigger();
   const int half = dh >> 1;
   const int heads = H + 2 * Hkv;
   const long long total = (long long)M * heads * half;
@@ -150,14 +150,12 @@ cudaError_t launch_qkv_finish(int dtype, const float* qkv, int n_split, long lon
   const int threads = 256;
   const int blocks = (int)std::min<long long>((total + threads - 1) / threads, 148LL * 16);
   if (dtype == kF32)
-    qkv_finish_kernel<float><<<blocks, threads, 0, s>>>(
-        qkv, n_split, split_stride, M, T, H, Hkv, dh, pos_base, cos_t, sin_t, max_pos,
-        (float*)q_out, (float*)k_cache, (float*)v_cache, t_max, err);
-  else
-    qkv_finish_kernel<bf16><<<blocks, threads, 0, s>>>(
-        qkv, n_split, split_stride, M, T, H, Hkv, dh, pos_base, cos_t, sin_t, max_pos,
-        (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, t_max, err);
-  return cudaGetLastError();
+    return launch_k(qkv_finish_kernel<float>, blocks, threads, 0, s, qkv, n_split, split_stride, M,
+                    T, H, Hkv, dh, pos_base, cos_t, sin_t, max_pos, (float*)q_out,
+                    (float*)k_cache, (float*)v_cache, t_max, err);
+  return launch_k(qkv_finish_kernel<bf16>, blocks, threads, 0, s, qkv, n_split, split_stride, M, T,
+                  H, Hkv, dh, pos_base, cos_t, sin_t, max_pos, (bf16*)q_out, (bf16*)k_cache,
+                  (bf16*)v_cache, t_max, err);
 }
 
 // ---------------------------------------------------------------- SiLU * up
@@ -168,6 +166,8 @@ cudaError_t launch_qkv_finish(int dtype, const float* qkv, int n_split, long lon
 template <typename T>
 __global__ void silu_mul_kernel(const float* __restrict__ gu, int n_split, long long split_stride,
                                 int M, int f, int n_packed, int block, T* __restrict__ a) {
+  pdl_wait();
+  pdl_trigger();
   const long long total = (long long)M * f;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
@@ -197,12 +197,10 @@ cudaError_t launch_silu_mul(int dtype, const float* gu, int n_split, long long s
   const int threads = 256;
   const int blocks = (int)std::min<long long>((total + threads - 1) / threads, 148LL * 16);
   if (dtype == kF32)
-    silu_mul_kernel<float><<<blocks, threads, 0, s>>>(gu, n_split, split_stride, M, f, n_packed,
-                                                      block, (float*)a);
-  else
-    silu_mul_kernel<bf16><<<blocks, threads, 0, s>>>(gu, n_split, split_stride, M, f, n_packed,
-                                                     block, (bf16*)a);
-  return cudaGetLastError();
+    return launch_k(silu_mul_kernel<float>, blocks, threads, 0, s, gu, n_split, split_stride, M, f,
+                    n_packed, block, (float*)a);
+  return launch_k(silu_mul_kernel<bf16>, blocks, threads, 0, s, gu, n_split, split_stride, M, f,
+                  n_packed, block, (bf16*)a);
 }
 
 // ---------------------------------------------------------------- residual add
@@ -212,6 +210,8 @@ template <typename T>
 __global__ void resid_add_kernel(const T* __restrict__ resid, const float* __restrict__ part,
                                  int n_split, long long split_stride, T* __restrict__ out,
                                  long long total, int* lens, int B, int len_inc) {
+  pdl_wait();
+  pdl_trigger();
   if (lens && blockIdx.x == 0)
     for (int b = threadIdx.x; b < B; b += blockDim.x) lens[b] += len_inc;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
@@ -229,25 +229,22 @@ cudaError_t launch_resid_add(int dtype, const void* resid, const float* part, in
   const int blocks =
       (int)std::max<long long>(1, std::min<long long>((total + threads - 1) / threads, 148LL * 16));
   if (dtype == kF32)
-    resid_add_kernel<float><<<blocks, threads, 0, s>>>((const float*)resid, part, n_split,
-                                                       split_stride, (float*)out, total, lens, B,
-                                                       len_inc);
-  else
-    resid_add_kernel<bf16><<<blocks, threads, 0, s>>>((const bf16*)resid, part, n_split,
-                                                      split_stride, (bf16*)out, total, lens, B,
-                                                      len_inc);
-  return cudaGetLastError();
+    return launch_k(resid_add_kernel<float>, blocks, threads, 0, s, (const float*)resid, part,
+                    n_split, split_stride, (float*)out, total, lens, B, len_inc);
+  return launch_k(resid_add_kernel<bf16>, blocks, threads, 0, s, (const bf16*)resid, part, n_split,
+                  split_stride, (bf16*)out, total, lens, B, len_inc);
 }
 
 // ---------------------------------------------------------------- lengths
 __global__ void set_lens_kernel(int* lens, int B, int value) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) lens[b] = value;
 }
 
 cudaError_t launch_set_lens(int* lens, int B, int value, cudaStream_t s) {
-  set_lens_kernel<<<(B + 127) / 128, 128, 0, s>>>(lens, B, value);
-  return cudaGetLastError();
+  return launch_k(set_lens_kernel, (B + 127) / 128, 128, 0, s, lens, B, value);
 }
 
 // ---------------------------------------------------------------- RoPE (standalone)
@@ -256,6 +253,7 @@ cudaError_t launch_set_lens(int* lens, int B, int value, cudaStream_t s) {
 template <typename T>
 __global__ void rope_apply_kernel(T* __restrict__ x, const int* __restrict__ pos, int B, int T_,
                                   int H, int dh, double base) {
+  pdl_wait();
   const int half = dh >> 1;
   const long long total = (long long)B * H * T_ * half;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;

@@ -6,6 +6,7 @@
 //     chapter 04.
 #include "common.cuh"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace lb {
 
@@ -22,6 +23,8 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
                                                        int N, int K) {
   __shared__ float As[kTK][kTM + 4];
   __shared__ float Bs[kTK][kTN + 4];
+  pdl_wait();
+  pdl_trigger();
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   const int m0 = blockIdx.y * kTM, n0 = blockIdx.x * kTN;
   float acc[4][4] = {};
@@ -67,8 +70,7 @@ cudaError_t launch_gemm_f32(const float* A, const float* B, float* C, const floa
                             int N, int K, cudaStream_t s) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   dim3 grid((N + kTN - 1) / kTN, (M + kTM - 1) / kTM);
-  gemm_f32_kernel<<<grid, 256, 0, s>>>(A, B, C, resid, M, N, K);
-  return cudaGetLastError();
+  return launch_k(gemm_f32_kernel, grid, 256, 0, s, A, B, C, resid, M, N, K);
 }
 
 // ---------------------------------------------------------------- attention
@@ -85,6 +87,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(
   __shared__ float qs[128];
   __shared__ float ps[kAttnThreads];
   __shared__ float red[32];
+  pdl_wait();
+  pdl_trigger();
   const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int hk = h / (H / Hkv);
   const int tk = kv_len ? kv_len[b] + 1 : Tk;
@@ -128,8 +132,8 @@ cudaError_t launch_attn_f32(const float* q, const float* k, const float* v, floa
                             const int* kv_len, cudaStream_t s) {
   if (B <= 0 || Tq <= 0) return cudaSuccess;
   dim3 grid(Tq, H, B);
-  attn_f32_kernel<<<grid, kAttnThreads, 0, s>>>(q, k, v, o, Tq, Tk, H, Hkv, dh, k_stride, kv_len);
-  return cudaGetLastError();
+  return launch_k(attn_f32_kernel, grid, kAttnThreads, 0, s, q, k, v, o, Tq, Tk, H, Hkv, dh,
+                  k_stride, kv_len);
 }
 
 }  // namespace lb

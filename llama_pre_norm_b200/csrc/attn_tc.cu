@@ -6,36 +6,43 @@
 // with GQA: query head h reads KV head h / (H / H_kv) (repeat_kv without
 // materialising the repeat).
 //
-// One CTA per (batch, head, 128-row query tile), heaviest tiles first. Key/value
-// tiles of 128 rows stream through a 2-stage TMA ring; tiles entirely above the
-// diagonal are never loaded, and the mask is applied only on tiles that cross it.
-//   warp 0      TMA producer (Q once, then K_j and V_j per tile)
-//   warp 1      TMEM allocation + single-thread MMA issue:
-//                 S_j = Q K_j^T into one of two TMEM score buffers (128 columns each),
-//                 O  += P_j V_j  into a TMEM accumulator (V read MN-major)
-//   warps 2..5  softmax: each thread owns one query row: reads its S row from
-//               TMEM, online max/sum in fp32 (base-2 exponent with log2(e)/sqrt(d_h)
-//               folded into the scale), rescales O in TMEM when the max moves,
-//               writes P (bf16) into shared memory in the MMA's swizzled K-major
-//               layout; finally O / l is written to o[b][t][h][:].
+// One CTA per (batch, head, pair of 128-row query tiles A and B), heaviest pairs
+// first. Both tiles consume the same 128-key K/V tiles, which stream through a
+// 2-stage TMA ring; K/V tiles above the diagonal are never loaded and the mask is
+// applied only on tiles that cross it.
+//   warp 0       TMA producer (Q_A, Q_B once; then K_j, V_j)
+//   warp 1       TMEM allocation + single-thread MMA issue, interleaving the tiles:
+//                  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), ...
+//                S_t = Q_t K_j^T lands in tile t's 128 score columns; the softmax
+//                writes P_t (bf16) over the first 64 of those columns and
+//                O_t += P_t V_j reads P_t straight from TMEM (V MN-major in smem).
+//                S_t(j+1) overwrites P_t(j), so it is issued only after PV_t(j) has
+//                completed; with two tiles in flight that wait leaves no bubble.
+//   warps 2..5   softmax of tile A, warps 6..9 softmax of tile B: one query row per
+//                thread (= TMEM lane); online max/sum in fp32 with ex2 and
+//                log2(e)/sqrt(d_h) folded into the scale. The running max is only
+//                moved (and O rescaled in TMEM) when a row's max grows by more than
+//                2^8, so most tiles skip the rescale; P <= 2^8 stays exact enough in
+//                bf16 and the final O / l uses the same reference max.
+// While one tile's softmax runs, the tensor core works on the other tile.
 #include "common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace lb {
 
-constexpr int kAttnTcThreads = 192;
+constexpr int kAttnTcThreads = 320;
+constexpr float kRescaleLog2 = 8.0f;
 
 template <int DH>
 struct AttnCfg {
   static constexpr int BQ = 128, BKV = 128;
-  static constexpr int PANELS = DH / 64;      // 64-column, 128-byte swizzled panels
+  static constexpr int PANELS = DH / 64;         // 64-column, 128-byte swizzled panels
   static constexpr int PANEL_BYTES = 128 * 128;  // one panel of a 128-row tile
   static constexpr int Q_BYTES = BQ * DH * 2;
   static constexpr int KV_BYTES = BKV * DH * 2;
-  static constexpr int P_BYTES = BQ * BKV * 2;
-  static constexpr int SMEM = Q_BYTES + 4 * KV_BYTES + P_BYTES + 256 + 1024;
-  static constexpr int TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256, 256+DH)
+  static constexpr int SMEM = 2 * Q_BYTES + 4 * KV_BYTES + 256 + 1024;
+  static constexpr int TMEM_COLS = 512;  // S/P of tile t at 128 t, O of tile t at 256 + 128 t
 };
 
 template <int DH>
@@ -47,32 +54,34 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + C::Q_BYTES;          // 2 stages
-  uint8_t* sV = sK + 2 * C::KV_BYTES;     // 2 stages
-  uint8_t* sP = sV + 2 * C::KV_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + C::P_BYTES);
+  uint8_t* sQ = smem;                      // tile A, then tile B
+  uint8_t* sK = sQ + 2 * C::Q_BYTES;       // 2 stages
+  uint8_t* sV = sK + 2 * C::KV_BYTES;      // 2 stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * C::KV_BYTES);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* v_full = bars + 3;    // [2]
-  uint64_t* kv_empty = bars + 5;  // [2]
-  uint64_t* s_full = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* o_full = bars + 10;
-  uint64_t* drain = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* k_full = bars + 1;    // [2 stages]
+  uint64_t* v_full = bars + 3;    // [2 stages]
+  uint64_t* kv_empty = bars + 5;  // [2 stages]
+  uint64_t* s_full = bars + 7;    // [2 tiles]
+  uint64_t* p_full = bars + 9;    // [2 tiles]
+  uint64_t* o_full = bars + 11;   // [2 tiles]
+  uint64_t* drain = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nq = (Tq + C::BQ - 1) / C::BQ;
+  const int npairs = (Tq + 2 * C::BQ - 1) / (2 * C::BQ);
   const int lin = blockIdx.x;
-  const int qt = nq - 1 - lin / (B * H);  // heaviest query tiles first
+  const int pr = npairs - 1 - lin / (B * H);  // heaviest pairs first
   const int bh = lin % (B * H);
   const int h = bh % H, b = bh / H;
   const int hk = h / (H / Hkv);
-  const int q0 = qt * C::BQ;
+  const int q0 = pr * 2 * C::BQ;
   const int off = Tk - Tq;  // query row i sits at position off + i
-  const int last_key = min(off + q0 + C::BQ - 1, Tk - 1);
-  const int n_kv = last_key / C::BKV + 1;
+  const bool hasB = q0 + C::BQ < Tq;
+  int n_t[2];
+  n_t[0] = min(off + q0 + C::BQ - 1, Tk - 1) / C::BKV + 1;
+  n_t[1] = hasB ? min(off + q0 + 2 * C::BQ - 1, Tk - 1) / C::BKV + 1 : 0;
+  const int n_max = max(n_t[0], n_t[1]);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -81,9 +90,9 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);  // one arrival per softmax warp of the tile
+      mbar_init(&o_full[i], 1);
     }
-    mbar_init(p_full, 4);  // one arrival per softmax warp
-    mbar_init(o_full, 1);
     mbar_init(drain, 1);
     fence_mbar_init();
     prefetch_tmap(&tmQ);
@@ -100,11 +109,13 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer
-      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
-      for (int p = 0; p < C::PANELS; ++p)
-        tma_load_3d(sQ + p * C::PANEL_BYTES, &tmQ, q_full, p * 64, q0, b * H + h);
+      mbar_arrive_expect_tx(q_full, (hasB ? 2 : 1) * C::Q_BYTES);
+      for (int t = 0; t < (hasB ? 2 : 1); ++t)
+        for (int p = 0; p < C::PANELS; ++p)
+          tma_load_3d(sQ + t * C::Q_BYTES + p * C::PANEL_BYTES, &tmQ, q_full, p * 64,
+                      q0 + t * C::BQ, b * H + h);
       int issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
+      for (int j = 0; j < n_max; ++j) {
         const int st = j & 1;
         if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1, err, 0x21)) break;
         mbar_arrive_expect_tx(&k_full[st], C::KV_BYTES);
@@ -130,67 +141,87 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
       // ---------------- MMA issuer
       constexpr uint32_t idesc_s = umma_idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_o = umma_idesc_bf16(128, DH, 0, 1);  // V is MN-major
-      const uint32_t q_addr = smem_u32(sQ);
-      bool ok = mbar_wait(q_full, 0, err, 0x23);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&k_full[st], (j >> 1) & 1, err, 0x24)) return false;
-        tc_fence_after();
+      auto issue_s = [&](int t, int st) {
+        const uint32_t q_addr = smem_u32(sQ + t * C::Q_BYTES);
         const uint32_t k_addr = smem_u32(sK + st * C::KV_BYTES);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t o = (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32;
-          umma_bf16(tmem_base + st * 128, umma_desc_sw128(q_addr + o, 16, 1024),
+          umma_bf16(tmem_base + t * 128, umma_desc_sw128(q_addr + o, 16, 1024),
                     umma_desc_sw128(k_addr + o, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[st]);
-        return true;
+        umma_commit(&s_full[t]);
       };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        if (j + 1 < n_kv && !issue_s(j + 1)) break;
-        if (!mbar_wait(p_full, j & 1, err, 0x25)) break;
-        const int st = j & 1;
-        if (!mbar_wait(&v_full[st], (j >> 1) & 1, err, 0x26)) break;
-        tc_fence_after();
-        const uint32_t p_addr = smem_u32(sP);
+      auto issue_pv = [&](int t, int st, int j) {
         const uint32_t v_addr = smem_u32(sV + st * C::KV_BYTES);
 #pragma unroll
         for (int kk = 0; kk < C::BKV / 16; ++kk) {
-          const uint64_t ad =
-              umma_desc_sw128(p_addr + (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32, 16, 1024);
-          // MN-major V: 16 keys = 16 rows of 128 B; the next 64 head dims are one
-          // panel (128 rows x 128 B) further.
+          // P_t: 8 TMEM columns per 16 keys. V: 16 keys = 16 rows of 128 B; the next
+          // 64 head dims are one panel (128 rows x 128 B) further.
           const uint64_t bd = umma_desc_sw128(v_addr + kk * 16 * 128, C::PANEL_BYTES, 1024);
-          umma_bf16(tmem_base + 256, ad, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a(tmem_base + 256 + t * 128, tmem_base + t * 128 + kk * 8, bd, idesc_o,
+                           (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&kv_empty[st]);
-        umma_commit(o_full);
+        umma_commit(&o_full[t]);
+      };
+      bool ok = mbar_wait(q_full, 0, err, 0x23) && mbar_wait(&k_full[0], 0, err, 0x24);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (n_t[t] > 0) issue_s(t, 0);
+      }
+      // Per tile: PV_t(j), then (once PV_t(j) has completed) S_t(j+1). Tile A's
+      // softmax of j+1 then overlaps tile B's PV(j) and S(j+1), and vice versa.
+      for (int j = 0; j < n_max && ok; ++j) {
+        const int st = j & 1;
+        bool v_ready = false, k_next_ready = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= n_t[t]) continue;
+          if (!mbar_wait(&p_full[t], j & 1, err, 0x25)) { ok = false; break; }
+          if (!v_ready && !mbar_wait(&v_full[st], (j >> 1) & 1, err, 0x26)) { ok = false; break; }
+          v_ready = true;
+          tc_fence_after();
+          issue_pv(t, st, j);
+          if (j + 1 < n_t[t]) {
+            if (!k_next_ready &&
+                !mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, err, 0x24)) { ok = false; break; }
+            k_next_ready = true;
+            // S_t(j+1) overwrites P_t(j): PV_t(j) must have completed
+            if (!mbar_wait(&o_full[t], j & 1, err, 0x27)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(t, (j + 1) & 1);
+          }
+        }
+        if (!ok) break;
+        umma_commit(&kv_empty[st]);  // K_j, V_j free once every MMA so far has completed
       }
       umma_commit(drain);
-      mbar_wait(drain, 0, err, 0x27);
+      mbar_wait(drain, 0, err, 0x28);
     }
   } else {
-    // ---------------- softmax / correction / output (warps 2..5)
+    // ---------------- softmax / correction / output (warps 2..5: tile A, 6..9: tile B)
+    const int t = (warp - 2) >> 2;
+    const int n = n_t[t];
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // query row within the tile == TMEM lane
-    const int qp = off + q0 + r;        // its position
-    const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t t_o = t_row + 256;
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(&s_full[st], (j >> 1) & 1, err, 0x28)) {
+    const int row0 = q0 + t * C::BQ;
+    const int qp = off + row0 + r;      // its position
+    const uint32_t lane_base = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t t_s = lane_base + t * 128;
+    const uint32_t t_o = lane_base + 256 + t * 128;
+    float m_ref = -INFINITY, l_run = 0.f;
+    bool ok = n > 0;
+    for (int j = 0; j < n && ok; ++j) {
+      if (!mbar_wait(&s_full[t], j & 1, err, 0x29)) {
         ok = false;
         break;
       }
       tc_fence_after();
       float s[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(t_row + st * 128 + c * 32, s[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, s[c]);
       tmem_wait_ld();
-      const bool need_mask = j * C::BKV + C::BKV - 1 > off + q0;
+      const bool need_mask = j * C::BKV + C::BKV - 1 > off + row0;
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -201,8 +232,11 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
           s[c][i] = v;
           mx = fmaxf(mx, v);
         }
-      const float m_new = fmaxf(m_run, mx);
-      const float alpha = ex2_approx(m_run - m_new);  // 0 on the first tile
+      // Move the reference max only when this row's max grew by more than 2^8
+      // (always on the first tile, where the reference is still -inf).
+      const bool move = mx > m_ref + kRescaleLog2;
+      const float m_new = move ? mx : m_ref;
+      const float alpha = move ? ex2_approx(m_ref - m_new) : 1.f;  // 0 on the first tile
       float rs = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -213,51 +247,47 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
           rs += p;
         }
       l_run = l_run * alpha + rs;
-      m_run = m_new;
-      if (j > 0) {
-        // P_{j-1} V_{j-1} must be complete: O is stable and the P buffer is free.
-        if (!mbar_wait(o_full, (j - 1) & 1, err, 0x29)) {
+      m_ref = m_new;
+      // P_t as bf16 pairs over the first 64 score columns (column c: keys 2c, 2c+1),
+      // packed in place: keys 0..63 into s[0], keys 64..127 into s[2].
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float* lo = s[2 * hh];
+        float* hi = s[2 * hh + 1];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) lo[i] = __uint_as_float(pack_bf16x2(lo[2 * i], lo[2 * i + 1]));
+#pragma unroll
+        for (int i = 0; i < 16; ++i) lo[16 + i] = __uint_as_float(pack_bf16x2(hi[2 * i], hi[2 * i + 1]));
+        tmem_st32(t_s + hh * 32, s[2 * hh]);
+      }
+      if (j > 0 && __any_sync(0xffffffffu, move)) {
+        // O_t holds PV_t(j-1) in full (S_t(j) was issued after it completed); it is
+        // rescaled before this tile's P is released to the MMA.
+        if (!mbar_wait(&o_full[t], (j - 1) & 1, err, 0x2a)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < DH / 32; ++c) {
-            float o[32];
-            tmem_ld32(t_o + c * 32, o);
-            tmem_wait_ld();
+        for (int c = 0; c < DH / 32; ++c) {
+          float o[32];
+          tmem_ld32(t_o + c * 32, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(t_o + c * 32, o);
-          }
-          tmem_wait_st();
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(t_o + c * 32, o);
         }
       }
-      // P row r into the swizzled K-major layout: key c -> panel c/64, 16-byte
-      // chunk (c%64)/8 stored at chunk ^ (r % 8).
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int c = ch >> 2, i0 = (ch & 3) * 8;
-        uint4 pk;
-        pk.x = pack_bf16x2(s[c][i0 + 0], s[c][i0 + 1]);
-        pk.y = pack_bf16x2(s[c][i0 + 2], s[c][i0 + 3]);
-        pk.z = pack_bf16x2(s[c][i0 + 4], s[c][i0 + 5]);
-        pk.w = pack_bf16x2(s[c][i0 + 6], s[c][i0 + 7]);
-        const int panel = ch >> 3, c16 = ch & 7;
-        *reinterpret_cast<uint4*>(sP + panel * C::PANEL_BYTES + r * 128 + ((c16 ^ (r & 7)) << 4)) =
-            pk;
-      }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    if (ok && mbar_wait(o_full, (n_kv - 1) & 1, err, 0x2a)) {
+    if (ok && mbar_wait(&o_full[t], (n - 1) & 1, err, 0x2b)) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
-      const bool store = q0 + r < Tq;
-      bf16* dst = out + (((long long)b * Tq + q0 + r) * H + h) * DH;
+      const bool store = row0 + r < Tq;
+      bf16* dst = out + (((long long)b * Tq + row0 + r) * H + h) * DH;
 #pragma unroll 1
       for (int c = 0; c < DH / 32; ++c) {
         float o[32];
@@ -266,10 +296,10 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
         if (store) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            float t[8];
+            float tt[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) t[i] = o[q * 8 + i] * inv_l;
-            store8(dst + c * 32 + q * 8, t);
+            for (int i = 0; i < 8; ++i) tt[i] = o[q * 8 + i] * inv_l;
+            store8(dst + c * 32 + q * 8, tt);
           }
         }
       }
@@ -300,10 +330,10 @@ static cudaError_t run_attn(const void* q, const void* k, const void* v, void* o
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int nq = (Tq + 127) / 128;
+  const int npairs = (Tq + 255) / 256;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
-  return launch_k(kern, nq * B * H, kAttnTcThreads, C::SMEM, s, tq, tk, tv, (bf16*)o, B, Tq, Tk, H,
-                  Hkv, scale_log2, err);
+  return launch_k(kern, npairs * B * H, kAttnTcThreads, C::SMEM, s, tq, tk, tv, (bf16*)o, B, Tq, Tk,
+                  H, Hkv, scale_log2, err);
 }
 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, int B, int Tq,

@@ -181,6 +181,7 @@ struct Carver {
 struct PrefillWs {
   void *h, *q, *o, *x1, *a;
   float *qkv32, *gu32;
+  float *ss1, *ss2;  // row sums of squares of X and X' (bf16 path)
 };
 struct DecodeWs {
   void *h, *q, *o, *x1, *a;
@@ -206,8 +207,11 @@ static PrefillWs carve_prefill(const llama_block* b, void* base, int M, size_t* 
   if (b->dtype == kF32) {
     w.qkv32 = (float*)c.take((size_t)M * b->n_qkv * 4);
     w.gu32 = (float*)c.take((size_t)M * b->n_gu * 4);
+    w.ss1 = w.ss2 = nullptr;
   } else {
     w.qkv32 = w.gu32 = nullptr;
+    w.ss1 = (float*)c.take((size_t)M * 4);
+    w.ss2 = (float*)c.take((size_t)M * 4);
   }
   *total = c.off;
   return w;
@@ -402,6 +406,12 @@ lb_status llama_block_set_weights(llama_block* b, const void* wq, const void* wk
                               cudaMemcpyDeviceToDevice, s));
     }
   }
+  if (b->dtype == kBF16) {
+    // RMSNorm gains folded into the weights that read the normalised rows:
+    // (g * x * r) W^T = r * x (W diag(g))^T; the GEMM epilogues apply r.
+    LB_CUDA(launch_scale_cols(b->w_qkv, g_attn, b->n_qkv, b->d, s));
+    LB_CUDA(launch_scale_cols(b->w_gu, g_mlp, b->n_gu, b->d, s));
+  }
   b->has_weights = true;
   return LB_OK;
 }
@@ -450,24 +460,26 @@ lb_status llama_block_prefill(llama_block* b, const void* x, void* y, int B, int
 
   b->stage_names.clear();
   if (b->dtype == kBF16) {
-    LB_STAGE("rmsnorm_attn", 1,
-             launch_resid_rmsnorm(kBF16, x, nullptr, 0, 0, nullptr, b->g1, w.h, M, d, b->eps, s));
+    // RMSNorm statistics of X (its gain is folded into W_qkv); also zeroes the X'
+    // statistic accumulated by o_proj and sets cache_len = T.
+    LB_STAGE("row_stats_attn", 1, launch_row_ssq(x, w.ss1, w.ss2, M, d, cache_len, B, T, s));
     GemmEpi e1;
     e1.kind = kEpiQkvRope;
     e1.T = T; e1.H = H; e1.Hkv = Hkv; e1.dh = dh; e1.t_max = t_max; e1.max_pos = b->max_pos;
     e1.q_out = w.q; e1.k_cache = k_cache; e1.v_cache = v_cache;
     e1.cos_t = b->cos_t; e1.sin_t = b->sin_t; e1.err = b->err;
-    LB_STAGE("qkv_rope_gemm", 1, launch_gemm_tc(w.h, b->w_qkv, M, b->n_qkv, d, 256, 1, e1, b->num_sms, s));
+    e1.row_ss = w.ss1; e1.row_inv_d = 1.f / d; e1.row_eps = b->eps;
+    LB_STAGE("qkv_rope_gemm", 1, launch_gemm_tc(x, b->w_qkv, M, b->n_qkv, d, 256, 1, e1, b->num_sms, s));
     LB_STAGE("attention", 1,
              launch_attn_tc(w.q, k_cache, v_cache, w.o, B, T, T, H, Hkv, dh, t_max, b->err, s));
     GemmEpi e2;
     e2.kind = kEpiResid; e2.out = w.x1; e2.resid = x; e2.ldo = d; e2.err = b->err;
+    e2.ss_out = w.ss2;  // statistic of X' for the MLP's RMSNorm
     LB_STAGE("o_proj_resid_gemm", 1, launch_gemm_tc(w.o, b->w_o, M, d, H * dh, 256, 1, e2, b->num_sms, s));
-    LB_STAGE("rmsnorm_mlp", 1,
-             launch_resid_rmsnorm(kBF16, w.x1, nullptr, 0, 0, nullptr, b->g2, w.h, M, d, b->eps, s));
     GemmEpi e3;
     e3.kind = kEpiSwiGLU; e3.out = w.a; e3.ldo = f; e3.f = f; e3.err = b->err;
-    LB_STAGE("gate_up_swiglu_gemm", 1, launch_gemm_tc(w.h, b->w_gu, M, b->n_gu, d, 256, 1, e3, b->num_sms, s));
+    e3.row_ss = w.ss2; e3.row_inv_d = 1.f / d; e3.row_eps = b->eps;
+    LB_STAGE("gate_up_swiglu_gemm", 1, launch_gemm_tc(w.x1, b->w_gu, M, b->n_gu, d, 256, 1, e3, b->num_sms, s));
     GemmEpi e4;
     e4.kind = kEpiResid; e4.out = y; e4.resid = w.x1; e4.ldo = d; e4.err = b->err;
     LB_STAGE("down_resid_gemm", 1, launch_gemm_tc(w.a, b->w_d, M, d, f, 256, 1, e4, b->num_sms, s));
@@ -492,8 +504,8 @@ lb_status llama_block_prefill(llama_block* b, const void* x, void* y, int B, int
     LB_STAGE("silu_mul", 1, launch_silu_mul(kF32, w.gu32, 1, 0, M, f, b->n_gu, 0, w.a, s));
     LB_STAGE("down_resid_gemm", 1, launch_gemm_f32((const float*)w.a, (const float*)b->w_d, (float*)y,
                                                    (const float*)w.x1, M, d, f, s));
+    LB_STAGE("set_lengths", 1, launch_set_lens(cache_len, B, T, s));
   }
-  LB_STAGE("set_lengths", 1, launch_set_lens(cache_len, B, T, s));
   b->lens.assign(B, T);
   return LB_OK;
 }
@@ -520,8 +532,9 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
   b->stage_names.clear();
   if (b->dtype == kBF16) {
     const int bn = B <= 32 ? 32 : B <= 64 ? 64 : B <= 128 ? 128 : 256;
+    // gains are folded into W_qkv / W_gu: the norms here only scale by 1/RMS
     LB_STAGE("rmsnorm_attn", 1,
-             launch_resid_rmsnorm(kBF16, x, nullptr, 0, 0, nullptr, b->g1, w.h, B, d, b->eps, s));
+             launch_resid_rmsnorm(kBF16, x, nullptr, 0, 0, nullptr, nullptr, w.h, B, d, b->eps, s));
     // Q|K|V: part[s][token][feature]
     GemmEpi e;
     e.kind = kEpiPartialT; e.out = w.part; e.err = b->err;
@@ -541,7 +554,7 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
     LB_STAGE("o_proj_gemm", 1, launch_gemm_tc(b->w_o, w.o, d, B, K2, bn, s2, e, b->num_sms, s));
     LB_STAGE("resid_rmsnorm_mlp", 1,
              launch_resid_rmsnorm(kBF16, x, w.part, gemm_effective_split(K2, s2), e.split_stride,
-                                  w.x1, b->g2, w.h, B, d, b->eps, s));
+                                  w.x1, nullptr, w.h, B, d, b->eps, s));
     // gate/up (packed rows), SiLU(g) * u
     const int s3 = decode_split((b->n_gu + 127) / 128, d);
     e.ldo = b->n_gu; e.split_stride = (long long)B * b->n_gu;

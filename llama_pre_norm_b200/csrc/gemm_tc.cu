@@ -57,6 +57,12 @@ __device__ __forceinline__ Unit decode_unit(int u, int num_m, int num_n, int KB,
 }
 
 // ------------------------------------------------------------------ epilogues
+// RMSNorm statistic of row m folded into the GEMM: rsqrt(mean square + eps), or 1.
+__device__ __forceinline__ float row_scale(const GemmEpi& e, int m, int M) {
+  if (!e.row_ss || m >= M) return 1.f;
+  return rsqrtf(e.row_ss[m] * e.row_inv_d + e.row_eps);
+}
+
 // Store 32 consecutive values of one output row at columns [n, n+32) of a row
 // with `ncols` columns: vectorised when the whole run is in range, else only
 // the in-range elements (ragged last tile).
@@ -79,6 +85,7 @@ __device__ __forceinline__ void epi_store_resid(uint32_t tb, int m, int nt, int 
                                                 const GemmEpi& e, bool with_resid) {
   bf16* out = reinterpret_cast<bf16*>(e.out);
   const bf16* res = reinterpret_cast<const bf16*>(e.resid);
+  float ssq = 0.f;
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     float v[32];
@@ -100,15 +107,24 @@ __device__ __forceinline__ void epi_store_resid(uint32_t tb, int m, int nt, int 
           for (int i = 0; i < 32 && n + i < N; ++i) v[i] += __bfloat162float(res[o + n + i]);
         }
       }
+      if (e.ss_out) {  // statistic of the stored (rounded) row for the next RMSNorm
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          v[i] = round_to<bf16>(v[i]);
+          if (n + i < N) ssq += v[i] * v[i];
+        }
+      }
       store_row32(out + o, n, N, v);
     }
   }
+  if (e.ss_out && m < M) atomicAdd(e.ss_out + m, ssq);
 }
 
 // Tile columns [0,128) are gate rows 128*nt.., [128,256) the matching up rows.
 __device__ __forceinline__ void epi_swiglu(uint32_t tb, int m, int nt, int M, int f,
                                            const GemmEpi& e) {
   bf16* out = reinterpret_cast<bf16*>(e.out);
+  const float r = row_scale(e, m, M);
 #pragma unroll 1
   for (int j = 0; j < 4; ++j) {
     float g[32], u[32];
@@ -118,7 +134,7 @@ __device__ __forceinline__ void epi_swiglu(uint32_t tb, int m, int nt, int M, in
     const int col = nt * 128 + j * 32;
     if (m < M && col < f) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
+      for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i] * r) * (u[i] * r);
       store_row32(out + (long long)m * e.ldo, col, f, g);
     }
   }
@@ -134,6 +150,7 @@ __device__ __forceinline__ void epi_qkv_rope(uint32_t tb, int m, int nt, int M, 
   const int b = m / e.T, t = m - (m / e.T) * e.T;
   const int pos = t;
   const bool row_ok = m < M;
+  const float r = row_scale(e, m, M);
   bool pos_ok = pos < e.max_pos && pos < e.t_max;
   if (row_ok && !pos_ok) latch_error(e.err, kErrCacheBounds);
 #pragma unroll 1
@@ -171,7 +188,7 @@ __device__ __forceinline__ void epi_qkv_rope(uint32_t tb, int m, int nt, int M, 
             load8(st + q * 8, s);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const float a = x1[q * 8 + i], bb = x2[q * 8 + i];
+              const float a = x1[q * 8 + i] * r, bb = x2[q * 8 + i] * r;
               o1[i] = a * c[i] - bb * s[i];
               o2[i] = bb * c[i] + a * s[i];
             }
@@ -191,7 +208,7 @@ __device__ __forceinline__ void epi_qkv_rope(uint32_t tb, int m, int nt, int M, 
           for (int q = 0; q < 4; ++q) {
             float o[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = x[q * 8 + i];
+            for (int i = 0; i < 8; ++i) o[i] = x[q * 8 + i] * r;
             store8(dst + j * 32 + q * 8, o);
           }
         }
@@ -372,6 +389,174 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ 2-SM pair kernel
+// The same GEMM with 256 x BN tiles computed by a cluster of two CTAs: CTA r of the
+// pair loads rows [128r, 128r+128) of the A tile and rows [r BN/2, (r+1) BN/2) of
+// the B tile into its own shared memory (32 KB per k-block at BN = 256, so six
+// stages fit), the even CTA issues tcgen05.mma.cta_group::2 (M = 256) which reads
+// both CTAs' operands and leaves each CTA's 128 accumulator rows in its own TMEM,
+// and both CTAs run the epilogue on their rows. Per SM the operand traffic per
+// MMA is two thirds of the 1-SM 128 x 256 tile's.
+template <int BN>
+struct Gemm2Cfg {
+  static constexpr int STAGES = 6;
+  static constexpr int A_BYTES = 128 * kBK * 2;
+  static constexpr int B_BYTES = (BN / 2) * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 256 + 1024;
+};
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, int M, int N, int K, GemmEpi epi) {
+  using C = Gemm2Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = bars;                  // used in the leader: both CTAs' bytes
+  uint64_t* empty = bars + C::STAGES;     // each CTA: its stage may be refilled
+  uint64_t* tfull = bars + 2 * C::STAGES; // each CTA: accumulator ready
+  uint64_t* tempty = tfull + 2;           // leader: both CTAs drained the accumulator
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA of the pair
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+
+  const int num_m = (M + 2 * kBM - 1) / (2 * kBM), num_n = (N + BN - 1) / BN;
+  const int KB = (K + kBK - 1) / kBK;
+  const int units = num_m * num_n;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs)
+      uint32_t stage = 0, phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int u = pair; u < units && ok; u += npairs) {
+        const int mt = u % num_m, nt = u / num_m;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, epi.err, 0x11)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          const uint32_t fb = pair_addr(&full[stage], 0);
+          tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, fb, kb * kBK, mt * 2 * kBM + rank * kBM);
+          tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, fb, kb * kBK, nt * BN + rank * (BN / 2));
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      pdl_trigger();
+      // The last loads must have landed and been consumed before the pair may exit.
+      const long long first = issued > C::STAGES ? issued - C::STAGES : 0;
+      for (long long i = first; i < issued; ++i)
+        mbar_wait(&empty[i % C::STAGES], (uint32_t)((i / C::STAGES) & 1), epi.err, 0x12);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (leader CTA)
+      constexpr uint32_t idesc = umma_idesc_bf16(2 * kBM, BN, 0, 0);
+      uint32_t stage = 0, phase = 0;
+      int t = 0;
+      bool ok = true;
+      for (int u = pair; u < units && ok; u += npairs, ++t) {
+        const int acc = t & 1;
+        if (!mbar_wait(&tempty[acc], ((t >> 1) & 1) ^ 1, epi.err, 0x13)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, epi.err, 0x14)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_bf16_pair(d_tmem, umma_desc_sw128(a0 + k * 32, 16, 1024),
+                           umma_desc_sw128(b0 + k * 32, 16, 1024), idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          umma_commit_pair(pair_addr(&empty[stage], 0));
+          umma_commit_pair(pair_addr(&empty[stage], 1));
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(pair_addr(&tfull[acc], 0));
+        umma_commit_pair(pair_addr(&tfull[acc], 1));
+      }
+      umma_commit_pair(pair_addr(drain, 0));
+      mbar_wait(drain, 0, epi.err, 0x15);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5 of both CTAs, 128 rows each)
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    int t = 0;
+    for (int u = pair; u < units; u += npairs, ++t) {
+      const int mt = u % num_m, nt = u / num_m;
+      const int acc = t & 1;
+      if (!mbar_wait(&tfull[acc], (t >> 1) & 1, epi.err, 0x16)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      const int m = mt * 2 * kBM + rank * kBM + row_in_tile;
+      if constexpr (EPI == kEpiStore) {
+        epi_store_resid<BN>(tb, m, nt, M, N, epi, false);
+      } else if constexpr (EPI == kEpiResid) {
+        epi_store_resid<BN>(tb, m, nt, M, N, epi, true);
+      } else if constexpr (EPI == kEpiSwiGLU) {
+        epi_swiglu(tb, m, nt, M, epi.f, epi);
+      } else {
+        epi_qkv_rope<BN>(tb, m, nt, M, N, epi);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(pair_addr(&tempty[acc], 0));
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();  // the leader's MMAs have finished reading both CTAs' operands
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 template <int BN, int EPI>
 static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
@@ -387,9 +572,43 @@ static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int M, int 
   return launch_k(kern, grid, kGemmThreads, C::SMEM, s, ta, tb, M, N, K, kb_per, n_split, epi);
 }
 
+template <int BN, int EPI>
+static cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
+                            const GemmEpi& epi, int grid, cudaStream_t s) {
+  using C = Gemm2Cfg<BN>;
+  auto kern = gemm_tc_pair_kernel<BN, EPI>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  return launch_k_pair(kern, grid, kGemmThreads, C::SMEM, s, ta, tb, M, N, K, epi);
+}
+
+// 2-SM pair path: 256 x 256 tiles, no split-K.
+static cudaError_t launch_gemm_tc_pair(const void* A, const void* B, int M, int N, int K,
+                                      const GemmEpi& epi, int num_sms, cudaStream_t s) {
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d_bf16(&ta, A, (uint64_t)M, (uint64_t)K, kBM)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d_bf16(&tb, B, (uint64_t)N, (uint64_t)K, 128)) return cudaErrorInvalidValue;
+  const long long units = (long long)((M + 255) / 256) * ((N + 255) / 256);
+  const int grid = (int)std::min<long long>(2 * units, num_sms & ~1);
+  switch (epi.kind) {
+    case kEpiStore: return run_pair<256, kEpiStore>(ta, tb, M, N, K, epi, grid, s);
+    case kEpiResid: return run_pair<256, kEpiResid>(ta, tb, M, N, K, epi, grid, s);
+    case kEpiSwiGLU: return run_pair<256, kEpiSwiGLU>(ta, tb, M, N, K, epi, grid, s);
+    case kEpiQkvRope: return run_pair<256, kEpiQkvRope>(ta, tb, M, N, K, epi, grid, s);
+  }
+  return cudaErrorInvalidConfiguration;
+}
+
 cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, int BN, int n_split,
                            const GemmEpi& epi, int num_sms, cudaStream_t s) {
   if (M <= 0 || N <= 0 || K <= 0) return cudaSuccess;
+  // Prefill-sized GEMMs run on CTA pairs (2-SM MMA, 256 x 256 tiles).
+  if (BN == 256 && n_split == 1 && epi.kind != kEpiPartialT && M > 128 && num_sms >= 2)
+    return launch_gemm_tc_pair(A, B, M, N, K, epi, num_sms, s);
   CUtensorMap ta, tb;
   if (!make_tmap_2d_bf16(&ta, A, (uint64_t)M, (uint64_t)K, kBM)) return cudaErrorInvalidValue;
   if (!make_tmap_2d_bf16(&tb, B, (uint64_t)N, (uint64_t)K, (uint32_t)BN))

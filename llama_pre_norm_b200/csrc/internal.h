@@ -49,6 +49,27 @@ inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
+// Same, launched as clusters of two CTAs (a 2-SM MMA pair); grid.x must be even.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k_pair(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ----------------------------------------------------------- norm_fuse.cu
 cudaError_t launch_resid_rmsnorm(int dtype, const void* x, const float* partial, int n_split,
                                  long long split_stride, void* x_out, const void* g, void* y,
@@ -63,6 +84,12 @@ cudaError_t launch_resid_add(int dtype, const void* resid, const float* part, in
                              long long split_stride, void* out, long long total, int* lens, int B,
                              int len_inc, cudaStream_t s);
 cudaError_t launch_set_lens(int* lens, int B, int value, cudaStream_t s);
+// ss[m] = sum_j x[m][j]^2 (fp32) for bf16 rows; zeroes ss_zero[m] (when given) for a
+// later accumulation; block 0 also sets lens[0..B) = len_value (when lens given).
+cudaError_t launch_row_ssq(const void* x, float* ss, float* ss_zero, int rows, int d, int* lens,
+                           int B, int len_value, cudaStream_t s);
+// w[r][c] = bf16(w[r][c] * g[c]) in place (bf16 [rows, cols], g [cols]).
+cudaError_t launch_scale_cols(void* w, const void* g, long long rows, int cols, cudaStream_t s);
 cudaError_t launch_rope_apply(int dtype, void* x, const int* pos, int B, int T, int H, int dh,
                               double base, cudaStream_t s);
 cudaError_t launch_selftest_timeout(int* err, unsigned long long budget_ns, cudaStream_t s);
@@ -101,6 +128,14 @@ struct GemmEpi {
   const float* cos_t = nullptr;
   const float* sin_t = nullptr;
   int* err = nullptr;
+  // RMSNorm folded into the GEMM (the gain is folded into the weights): when
+  // row_ss != NULL the accumulator of row m is multiplied by
+  // rsqrt(row_ss[m] * row_inv_d + row_eps) before the epilogue op (QkvRope, SwiGLU).
+  const float* row_ss = nullptr;
+  float row_inv_d = 0.f, row_eps = 0.f;
+  // kEpiResid: when ss_out != NULL, the sum of squares of each stored (rounded)
+  // output row is accumulated into ss_out[m] (atomically, over the N tiles).
+  float* ss_out = nullptr;
 };
 
 // D[M,N] = A[M,K] · B[N,K]^T, bf16 operands (K-major, row stride K), fp32 accumulation in

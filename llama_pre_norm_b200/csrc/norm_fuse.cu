@@ -19,7 +19,8 @@ namespace lb {
 // ---------------------------------------------------------------- RMSNorm
 // One CTA per row. x_row = resid[row] + sum_s partial[s][row] (fp32), rounded to
 // T; if x_out: stored there (the residual stream X'). y = g * x_row * r,
-// r = 1/sqrt(mean(x_row^2) + eps), computed in fp32, rounded once.
+// r = 1/sqrt(mean(x_row^2) + eps), computed in fp32, rounded once (g == NULL:
+// the gain has been folded into the next GEMM's weights, y = x_row * r).
 // Each thread keeps up to kMaxVec 8-element vectors of the row in registers.
 constexpr int kNormThreads = 256;
 constexpr int kMaxVec = 4;  // rows up to 256 * 8 * 4 = 8192 elements
@@ -61,7 +62,12 @@ __global__ void __launch_bounds__(kNormThreads) resid_rmsnorm_kernel(
     const int vi = threadIdx.x + i * kNormThreads;
     if (vi < nvec) {
       float gg[8], o[8];
-      load8(g + vi * 8, gg);
+      if (g) {
+        load8(g + vi * 8, gg);
+      } else {  // gain folded into the consumer's weights
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gg[e] = 1.f;
+      }
 #pragma unroll
       for (int e = 0; e < 8; ++e) o[e] = gg[e] * (v[i][e] * r);
       store8(y + row * d + vi * 8, o);
@@ -233,6 +239,72 @@ cudaError_t launch_resid_add(int dtype, const void* resid, const float* part, in
                     n_split, split_stride, (float*)out, total, lens, B, len_inc);
   return launch_k(resid_add_kernel<bf16>, blocks, threads, 0, s, (const bf16*)resid, part, n_split,
                   split_stride, (bf16*)out, total, lens, B, len_inc);
+}
+
+// ---------------------------------------------------------------- row statistics
+// Sum of squares of each bf16 row (the RMSNorm statistic; the GEMM that consumes
+// the row applies rsqrt(ss/d + eps) in its epilogue). One warp per row with all
+// of the row's 16-byte loads issued before the first use, so each SM keeps many
+// loads in flight.
+constexpr int kSsqWarps = 8;
+constexpr int kSsqMaxVec = 32;  // 16-byte vectors per lane: rows up to 32*8*32 = 8192
+
+__global__ void __launch_bounds__(kSsqWarps * 32) row_ssq_kernel(const bf16* __restrict__ x,
+                                                                 float* __restrict__ ss,
+                                                                 float* __restrict__ ss_zero,
+                                                                 int rows, int d, int* lens, int B,
+                                                                 int len_value) {
+  pdl_wait();
+  pdl_trigger();
+  if (lens && blockIdx.x == 0)
+    for (int b = threadIdx.x; b < B; b += blockDim.x) lens[b] = len_value;
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kSsqWarps + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int nvec = d >> 3;
+  const uint4* src = reinterpret_cast<const uint4*>(x + row * d);
+  uint4 u[kSsqMaxVec];
+#pragma unroll
+  for (int i = 0; i < kSsqMaxVec; ++i)
+    if (lane + 32 * i < nvec) u[i] = src[lane + 32 * i];
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < kSsqMaxVec; ++i) {
+    if (lane + 32 * i < nvec) {
+      float v[8];
+      unpack_bf16x8(u[i], v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc = fmaf(v[e], v[e], acc);
+    }
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) {
+    ss[row] = acc;
+    if (ss_zero) ss_zero[row] = 0.f;
+  }
+}
+
+cudaError_t launch_row_ssq(const void* x, float* ss, float* ss_zero, int rows, int d, int* lens,
+                           int B, int len_value, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  return launch_k(row_ssq_kernel, (rows + kSsqWarps - 1) / kSsqWarps, kSsqWarps * 32, 0, s,
+                  (const bf16*)x, ss, ss_zero, rows, d, lens, B, len_value);
+}
+
+// Fold an RMSNorm gain into the weights that consume the normalised row:
+// (g * x * r) W^T = r * x (W diag(g))^T.
+__global__ void scale_cols_kernel(bf16* __restrict__ w, const bf16* __restrict__ g, long long rows,
+                                  int cols) {
+  pdl_wait();
+  const long long total = rows * cols;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x)
+    w[i] = __float2bfloat16_rn(__bfloat162float(w[i]) * __bfloat162float(g[i % cols]));
+}
+
+cudaError_t launch_scale_cols(void* w, const void* g, long long rows, int cols, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  return launch_k(scale_cols_kernel, 148 * 16, 256, 0, s, (bf16*)w, (const bf16*)g, rows, cols);
 }
 
 // ---------------------------------------------------------------- lengths

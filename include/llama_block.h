@@ -103,6 +103,18 @@ lb_status llama_block_decode(llama_block* blk, const void* x, void* y, int B,
                              void* k_cache, void* v_cache, int t_max, int32_t* cache_len,
                              void* stream);
 
+/* Chunked prefill into an existing cache (mechanics page, chapter 04: the prefill ->
+ * decode handoff; positions follow the cache length). Every sequence must hold the
+ * same number L of cached tokens (host mirror: prefill, extend, decode or
+ * llama_block_set_lengths), else LB_ERR_UNSUPPORTED. The T new tokens x [B, T, d]
+ * sit at positions L .. L+T-1: their rotated keys and values are written to cache
+ * indices L .. L+T-1, token i attends to keys 0 .. L+i, y [B, T, d] is the block
+ * output, and cache_len becomes L + T. L + T <= t_max and <= max_pos required (else
+ * LB_ERR_CACHE_FULL). With L = 0 this is llama_block_prefill. */
+lb_status llama_block_extend(llama_block* blk, const void* x, void* y, int B, int T,
+                             void* k_cache, void* v_cache, int t_max, int32_t* cache_len,
+                             void* stream);
+
 /* Tell the handle the current cache lengths (host array of B entries) when the
  * caller filled the cache itself; the device cache_len array stays the caller's
  * to set. */
@@ -149,6 +161,44 @@ unsigned long long llama_block_launch_count(const llama_block* blk);
  * llama_block_sync_status(NULL, stream) then returns LB_ERR_TIMEOUT. No GPU fault
  * or hang is involved. */
 lb_status llama_block_selftest_timeout(long long budget_ns, void* stream);
+
+/* ---------------- stack of blocks ---------------- */
+
+/* A stack of n_layers decoder blocks with the same shape (mechanics page, chapter 02:
+ * the block repeated "x L"; LMDrive page §1: 32 decoder layers), each with its own
+ * weights and KV cache; layer l's output feeds layer l+1. The stack owns its layer
+ * handles, two activation buffers [B*T, d] and per-layer length arrays; the caller
+ * owns the caches. */
+typedef struct llama_stack llama_stack;
+
+lb_status llama_stack_create(int n_layers, int d, int n_heads, int n_kv_heads, int head_dim,
+                             int f, float eps, float rope_base, lb_dtype dtype, int max_pos,
+                             llama_stack** out);
+
+/* The block handle of layer `layer` (for llama_block_set_weights); NULL when out of
+ * range. Owned by the stack. */
+llama_block* llama_stack_layer(llama_stack* st, int layer);
+
+/* Prefill / chunked prefill / one decode step through every layer. k_caches and
+ * v_caches are HOST arrays of n_layers device pointers, each cache
+ * [B, n_kv_heads, t_max, head_dim]. cache_len (device int32 [B]) is read at the
+ * start and holds the new lengths at the end, as for a single block. x, y as for
+ * the block calls (T = 1 for decode). */
+lb_status llama_stack_prefill(llama_stack* st, const void* x, void* y, int B, int T,
+                              void* const* k_caches, void* const* v_caches, int t_max,
+                              int32_t* cache_len, void* stream);
+lb_status llama_stack_extend(llama_stack* st, const void* x, void* y, int B, int T,
+                             void* const* k_caches, void* const* v_caches, int t_max,
+                             int32_t* cache_len, void* stream);
+lb_status llama_stack_decode(llama_stack* st, const void* x, void* y, int B,
+                             void* const* k_caches, void* const* v_caches, int t_max,
+                             int32_t* cache_len, void* stream);
+
+/* Set the host length mirror of every layer (see llama_block_set_lengths). */
+lb_status llama_stack_set_lengths(llama_stack* st, const int32_t* lens_host, int B);
+
+/* Free the stack, its layers and its buffers. */
+void llama_stack_destroy(llama_stack* st);
 
 /* ---------------- standalone entry points (testing) ---------------- */
 

@@ -19,11 +19,13 @@ import torch
 __all__ = [
     "LB_F32", "LB_BF16", "LlamaBlockError", "lib", "lib_path", "dtype_code",
     "llama_block_create", "llama_block_set_weights", "llama_block_reserve",
-    "llama_block_prefill", "llama_block_decode", "llama_block_set_lengths",
+    "llama_block_prefill", "llama_block_extend", "llama_block_decode", "llama_block_set_lengths",
     "llama_block_kv_cache_bytes", "llama_block_sync_status", "llama_block_destroy",
     "llama_block_last_error", "llama_block_selftest_timeout", "llama_block_enable_timing",
     "llama_block_stage_times", "llama_block_stage_name", "llama_block_launch_count",
     "rmsnorm", "rope_apply", "causal_attn", "swiglu_mlp", "decode_attn_static_scratch", "LlamaBlock",
+    "llama_stack_create", "llama_stack_layer", "llama_stack_prefill", "llama_stack_extend",
+    "llama_stack_decode", "llama_stack_set_lengths", "llama_stack_destroy", "LlamaStack",
 ]
 
 LB_F32, LB_BF16 = 0, 1
@@ -44,7 +46,15 @@ _SIGS = {
     "llama_block_set_weights": (_i, [_p] * 11),
     "llama_block_reserve": (_i, [_p, _i, _i]),
     "llama_block_prefill": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p]),
+    "llama_block_extend": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p]),
     "llama_block_decode": (_i, [_p, _p, _p, _i, _p, _p, _i, _p, _p]),
+    "llama_stack_create": (_i, [_i, _i, _i, _i, _i, _i, _f, _f, _i, _i, _pp]),
+    "llama_stack_layer": (_p, [_p, _i]),
+    "llama_stack_prefill": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p]),
+    "llama_stack_extend": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p]),
+    "llama_stack_decode": (_i, [_p, _p, _p, _i, _p, _p, _i, _p, _p]),
+    "llama_stack_set_lengths": (_i, [_p, _p, _i]),
+    "llama_stack_destroy": (None, [_p]),
     "llama_block_set_lengths": (_i, [_p, _p, _i]),
     "llama_block_kv_cache_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "llama_block_sync_status": (_i, [_p, _p]),
@@ -136,6 +146,15 @@ def llama_block_prefill(h, x, y, k_cache, v_cache, cache_len, stream=None):
                                    _ptr(k_cache, "k_cache", x.dtype), _ptr(v_cache, "v_cache", x.dtype),
                                    t_max, _ptr(cache_len, "cache_len", torch.int32), _stream(stream)),
            "llama_block_prefill")
+
+
+def llama_block_extend(h, x, y, k_cache, v_cache, cache_len, stream=None):
+    B, T, _ = x.shape
+    t_max = k_cache.shape[2]
+    _check(lib.llama_block_extend(h, _ptr(x, "x"), _ptr(y, "y", x.dtype), B, T,
+                                  _ptr(k_cache, "k_cache", x.dtype), _ptr(v_cache, "v_cache", x.dtype),
+                                  t_max, _ptr(cache_len, "cache_len", torch.int32), _stream(stream)),
+           "llama_block_extend")
 
 
 def llama_block_decode(h, x, y, k_cache, v_cache, cache_len, stream=None):
@@ -258,6 +277,9 @@ class LlamaBlock:
     def prefill(self, x, y, k_cache, v_cache, cache_len, stream=None):
         llama_block_prefill(self.handle, x, y, k_cache, v_cache, cache_len, stream)
 
+    def extend(self, x, y, k_cache, v_cache, cache_len, stream=None):
+        llama_block_extend(self.handle, x, y, k_cache, v_cache, cache_len, stream)
+
     def decode(self, x, y, k_cache, v_cache, cache_len, stream=None):
         llama_block_decode(self.handle, x, y, k_cache, v_cache, cache_len, stream)
 
@@ -280,6 +302,100 @@ class LlamaBlock:
     def close(self):
         if self.handle:
             llama_block_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ----------------------------------------------------------------- stack of blocks
+def _ptr_array(ts, name, dtype):
+    arr = (ctypes.c_void_p * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = _ptr(t, f"{name}[{i}]", dtype)
+    return arr
+
+
+def llama_stack_create(n_layers, d, n_heads, n_kv_heads, head_dim, f, eps, rope_base, dtype, max_pos) -> int:
+    out = ctypes.c_void_p()
+    code = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    _check(lib.llama_stack_create(n_layers, d, n_heads, n_kv_heads, head_dim, f, eps, rope_base, code,
+                                  max_pos, ctypes.byref(out)), "llama_stack_create")
+    return out.value
+
+
+def llama_stack_layer(st, layer) -> int:
+    h = lib.llama_stack_layer(st, layer)
+    if not h:
+        raise IndexError(f"layer {layer} out of range")
+    return h
+
+
+def _stack_call(fn, name, st, x, y, k_caches, v_caches, cache_len, stream, with_T=True):
+    B, T = x.shape[0], x.shape[1]
+    t_max = k_caches[0].shape[2]
+    args = [st, _ptr(x, "x"), _ptr(y, "y", x.dtype), B]
+    if with_T:
+        args.append(T)
+    args += [_ptr_array(k_caches, "k_caches", x.dtype), _ptr_array(v_caches, "v_caches", x.dtype), t_max,
+             _ptr(cache_len, "cache_len", torch.int32), _stream(stream)]
+    _check(fn(*args), name)
+
+
+def llama_stack_prefill(st, x, y, k_caches, v_caches, cache_len, stream=None):
+    _stack_call(lib.llama_stack_prefill, "llama_stack_prefill", st, x, y, k_caches, v_caches, cache_len, stream)
+
+
+def llama_stack_extend(st, x, y, k_caches, v_caches, cache_len, stream=None):
+    _stack_call(lib.llama_stack_extend, "llama_stack_extend", st, x, y, k_caches, v_caches, cache_len, stream)
+
+
+def llama_stack_decode(st, x, y, k_caches, v_caches, cache_len, stream=None):
+    _stack_call(lib.llama_stack_decode, "llama_stack_decode", st, x, y, k_caches, v_caches, cache_len, stream,
+                with_T=False)
+
+
+def llama_stack_set_lengths(st, lens):
+    arr = (ctypes.c_int32 * len(lens))(*[int(v) for v in lens])
+    _check(lib.llama_stack_set_lengths(st, arr, len(lens)), "llama_stack_set_lengths")
+
+
+def llama_stack_destroy(st):
+    lib.llama_stack_destroy(st)
+
+
+class LlamaStack:
+    """Owns a ``llama_stack`` of n_layers blocks (per-layer weights and caches)."""
+
+    def __init__(self, n_layers, d, n_heads, n_kv_heads, head_dim, f, eps=1e-6, rope_base=10000.0,
+                 dtype=torch.bfloat16, max_pos=4096):
+        self.n_layers = n_layers
+        self.handle = llama_stack_create(n_layers, d, n_heads, n_kv_heads, head_dim, f, eps, rope_base,
+                                         dtype_code(dtype), max_pos)
+
+    def set_layer_weights(self, layer, w: dict, stream=None):
+        h = llama_stack_layer(self.handle, layer)
+        llama_block_set_weights(h, w["wq"], w["wk"], w["wv"], w["wo"], w["w_gate"], w["w_up"],
+                                w["w_down"], w["g_attn"], w["g_mlp"], stream)
+
+    def prefill(self, x, y, k_caches, v_caches, cache_len, stream=None):
+        llama_stack_prefill(self.handle, x, y, k_caches, v_caches, cache_len, stream)
+
+    def extend(self, x, y, k_caches, v_caches, cache_len, stream=None):
+        llama_stack_extend(self.handle, x, y, k_caches, v_caches, cache_len, stream)
+
+    def decode(self, x, y, k_caches, v_caches, cache_len, stream=None):
+        llama_stack_decode(self.handle, x, y, k_caches, v_caches, cache_len, stream)
+
+    def set_lengths(self, lens):
+        llama_stack_set_lengths(self.handle, lens)
+
+    def close(self):
+        if self.handle:
+            llama_stack_destroy(self.handle)
             self.handle = None
 
     def __del__(self):

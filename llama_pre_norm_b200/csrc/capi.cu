@@ -442,15 +442,12 @@ static lb_status check_cache_args(llama_block* b, const void* x, const void* y, 
   return LB_OK;
 }
 
-lb_status llama_block_prefill(llama_block* b, const void* x, void* y, int B, int T, void* k_cache,
-                              void* v_cache, int t_max, int32_t* cache_len, void* stream) {
-  lb_status st = check_cache_args(b, x, y, B, k_cache, v_cache, t_max, cache_len, "prefill");
-  if (st != LB_OK) return st;
-  if (T <= 0) return fail(LB_ERR_INVALID_ARG, "prefill: T must be positive");
-  if (T > t_max || T > b->max_pos)
-    return fail(LB_ERR_CACHE_FULL, "prefill: T=%d exceeds t_max=%d or max_pos=%d", T, t_max,
-                b->max_pos);
-  cudaStream_t s = (cudaStream_t)stream;
+// Prefill of T tokens per sequence appended at cache position L (L = 0: a fresh
+// prefill; L > 0: chunked prefill into an existing cache).
+static lb_status run_prefill(llama_block* b, const void* x, void* y, int B, int T, int L,
+                             void* k_cache, void* v_cache, int t_max, int32_t* cache_len,
+                             cudaStream_t s) {
+  lb_status st;
   const int M = B * T;
   size_t need = 0;
   carve_prefill(b, nullptr, M, &need);
@@ -461,17 +458,17 @@ lb_status llama_block_prefill(llama_block* b, const void* x, void* y, int B, int
   b->stage_names.clear();
   if (b->dtype == kBF16) {
     // RMSNorm statistics of X (its gain is folded into W_qkv); also zeroes the X'
-    // statistic accumulated by o_proj and sets cache_len = T.
-    LB_STAGE("row_stats_attn", 1, launch_row_ssq(x, w.ss1, w.ss2, M, d, cache_len, B, T, s));
+    // statistic accumulated by o_proj and sets cache_len = L + T.
+    LB_STAGE("row_stats_attn", 1, launch_row_ssq(x, w.ss1, w.ss2, M, d, cache_len, B, L + T, s));
     GemmEpi e1;
     e1.kind = kEpiQkvRope;
     e1.T = T; e1.H = H; e1.Hkv = Hkv; e1.dh = dh; e1.t_max = t_max; e1.max_pos = b->max_pos;
-    e1.q_out = w.q; e1.k_cache = k_cache; e1.v_cache = v_cache;
+    e1.q_out = w.q; e1.k_cache = k_cache; e1.v_cache = v_cache; e1.pos0 = L;
     e1.cos_t = b->cos_t; e1.sin_t = b->sin_t; e1.err = b->err;
     e1.row_ss = w.ss1; e1.row_inv_d = 1.f / d; e1.row_eps = b->eps;
     LB_STAGE("qkv_rope_gemm", 1, launch_gemm_tc(x, b->w_qkv, M, b->n_qkv, d, 256, 1, e1, b->num_sms, s));
     LB_STAGE("attention", 1,
-             launch_attn_tc(w.q, k_cache, v_cache, w.o, B, T, T, H, Hkv, dh, t_max, b->err, s));
+             launch_attn_tc(w.q, k_cache, v_cache, w.o, B, T, L + T, H, Hkv, dh, t_max, b->err, s));
     GemmEpi e2;
     e2.kind = kEpiResid; e2.out = w.x1; e2.resid = x; e2.ldo = d; e2.err = b->err;
     e2.ss_out = w.ss2;  // statistic of X' for the MLP's RMSNorm
@@ -489,12 +486,12 @@ lb_status llama_block_prefill(llama_block* b, const void* x, void* y, int B, int
              launch_resid_rmsnorm(kF32, x, nullptr, 0, 0, nullptr, b->g1, w.h, M, d, b->eps, s));
     LB_STAGE("qkv_gemm", 1, launch_gemm_f32((const float*)w.h, (const float*)b->w_qkv, w.qkv32, nullptr, M,
                                             b->n_qkv, d, s));
-    LB_STAGE("qkv_rope", 1, launch_qkv_finish(kF32, w.qkv32, 1, 0, M, T, H, Hkv, dh, nullptr, b->cos_t,
+    LB_STAGE("qkv_rope", 1, launch_qkv_finish(kF32, w.qkv32, 1, 0, M, T, H, Hkv, dh, nullptr, L, b->cos_t,
                                               b->sin_t, b->max_pos, w.q, k_cache, v_cache, t_max,
                                               b->err, s));
     LB_STAGE("attention", 1, launch_attn_f32((const float*)w.q, (const float*)k_cache,
-                                             (const float*)v_cache, (float*)w.o, B, T, T, H, Hkv, dh,
-                                             t_max, nullptr, s));
+                                             (const float*)v_cache, (float*)w.o, B, T, L + T, H, Hkv,
+                                             dh, t_max, nullptr, s));
     LB_STAGE("o_proj_resid_gemm", 1, launch_gemm_f32((const float*)w.o, (const float*)b->w_o,
                                                      (float*)w.x1, X, M, d, H * dh, s));
     LB_STAGE("rmsnorm_mlp", 1,
@@ -504,10 +501,40 @@ lb_status llama_block_prefill(llama_block* b, const void* x, void* y, int B, int
     LB_STAGE("silu_mul", 1, launch_silu_mul(kF32, w.gu32, 1, 0, M, f, b->n_gu, 0, w.a, s));
     LB_STAGE("down_resid_gemm", 1, launch_gemm_f32((const float*)w.a, (const float*)b->w_d, (float*)y,
                                                    (const float*)w.x1, M, d, f, s));
-    LB_STAGE("set_lengths", 1, launch_set_lens(cache_len, B, T, s));
+    LB_STAGE("set_lengths", 1, launch_set_lens(cache_len, B, L + T, s));
   }
-  b->lens.assign(B, T);
+  b->lens.assign(B, L + T);
   return LB_OK;
+}
+
+lb_status llama_block_prefill(llama_block* b, const void* x, void* y, int B, int T, void* k_cache,
+                              void* v_cache, int t_max, int32_t* cache_len, void* stream) {
+  lb_status st = check_cache_args(b, x, y, B, k_cache, v_cache, t_max, cache_len, "prefill");
+  if (st != LB_OK) return st;
+  if (T <= 0) return fail(LB_ERR_INVALID_ARG, "prefill: T must be positive");
+  if (T > t_max || T > b->max_pos)
+    return fail(LB_ERR_CACHE_FULL, "prefill: T=%d exceeds t_max=%d or max_pos=%d", T, t_max,
+                b->max_pos);
+  return run_prefill(b, x, y, B, T, 0, k_cache, v_cache, t_max, cache_len, (cudaStream_t)stream);
+}
+
+lb_status llama_block_extend(llama_block* b, const void* x, void* y, int B, int T, void* k_cache,
+                             void* v_cache, int t_max, int32_t* cache_len, void* stream) {
+  lb_status st = check_cache_args(b, x, y, B, k_cache, v_cache, t_max, cache_len, "extend");
+  if (st != LB_OK) return st;
+  if (T <= 0) return fail(LB_ERR_INVALID_ARG, "extend: T must be positive");
+  if ((int)b->lens.size() != B)
+    return fail(LB_ERR_INVALID_ARG,
+                "extend: the handle knows %d sequence lengths, B=%d (call prefill or set_lengths)",
+                (int)b->lens.size(), B);
+  const int L = b->lens[0];
+  for (int i = 1; i < B; ++i)
+    if (b->lens[i] != L)
+      return fail(LB_ERR_UNSUPPORTED, "extend: the sequences have different cache lengths");
+  if (L < 0 || L + T > t_max || L + T > b->max_pos)
+    return fail(LB_ERR_CACHE_FULL, "extend: length %d + %d exceeds t_max=%d or max_pos=%d", L, T,
+                t_max, b->max_pos);
+  return run_prefill(b, x, y, B, T, L, k_cache, v_cache, t_max, cache_len, (cudaStream_t)stream);
 }
 
 lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void* k_cache,
@@ -543,7 +570,7 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
     LB_STAGE("qkv_gemm", 1, launch_gemm_tc(b->w_qkv, w.h, b->n_qkv, B, d, bn, s1, e, b->num_sms, s));
     LB_STAGE("qkv_rope_append", 1,
              launch_qkv_finish(kBF16, w.part, gemm_effective_split(d, s1), e.split_stride, B, 1, H,
-                               Hkv, dh, cache_len, b->cos_t, b->sin_t, b->max_pos, w.q, k_cache,
+                               Hkv, dh, cache_len, 0, b->cos_t, b->sin_t, b->max_pos, w.q, k_cache,
                                v_cache, t_max, b->err, s));
     LB_STAGE("attention", 2, launch_attn_decode(w.q, k_cache, v_cache, w.o, w.attn_part, B, H, Hkv,
                                                 dh, t_max, cache_len, b->err, s));
@@ -575,7 +602,7 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
     LB_STAGE("qkv_gemm", 1, launch_gemm_f32((const float*)w.h, (const float*)b->w_qkv, w.part, nullptr,
                                             B, b->n_qkv, d, s));
     LB_STAGE("qkv_rope_append", 1,
-             launch_qkv_finish(kF32, w.part, 1, 0, B, 1, H, Hkv, dh, cache_len, b->cos_t, b->sin_t,
+             launch_qkv_finish(kF32, w.part, 1, 0, B, 1, H, Hkv, dh, cache_len, 0, b->cos_t, b->sin_t,
                                b->max_pos, w.q, k_cache, v_cache, t_max, b->err, s));
     LB_STAGE("attention", 1, launch_attn_f32((const float*)w.q, (const float*)k_cache,
                                              (const float*)v_cache, (float*)w.o, B, 1, 1, H, Hkv, dh,
@@ -761,6 +788,154 @@ lb_status swiglu_mlp(const void* h, const void* w_gate, const void* w_up, const 
   st = run();
   cudaFreeAsync(tmp, s);
   return st;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ stack of blocks
+// L decoder layers applied in sequence (the "x L blocks" of the mechanics page's
+// chapter-02 diagram; LMDrive page §1, 32 LlamaDecoderLayers). Each layer is a
+// llama_block with its own weights and its own caller-owned KV cache; the stack
+// owns two ping-pong activation buffers and one device length array per layer.
+struct llama_stack {
+  std::vector<llama_block*> layers;
+  int d = 0;
+  size_t esz = 0;
+  void* act[2] = {nullptr, nullptr};
+  size_t act_bytes = 0;
+  int32_t* lens = nullptr;  // [layers][B]
+  int lens_cap = 0;
+};
+
+extern "C" {
+
+void llama_stack_destroy(llama_stack* st) {
+  if (!st) return;
+  cudaDeviceSynchronize();
+  for (llama_block* b : st->layers) llama_block_destroy(b);
+  for (void* p : {st->act[0], st->act[1], (void*)st->lens})
+    if (p) cudaFree(p);
+  delete st;
+}
+
+lb_status llama_stack_create(int n_layers, int d, int n_heads, int n_kv_heads, int head_dim, int f,
+                             float eps, float rope_base, lb_dtype dtype, int max_pos,
+                             llama_stack** out) {
+  if (!out) return fail(LB_ERR_INVALID_ARG, "stack_create: out is NULL");
+  *out = nullptr;
+  if (n_layers <= 0) return fail(LB_ERR_INVALID_ARG, "stack_create: n_layers must be positive");
+  llama_stack* st = new llama_stack();
+  for (int l = 0; l < n_layers; ++l) {
+    llama_block* b = nullptr;
+    const lb_status r =
+        llama_block_create(d, n_heads, n_kv_heads, head_dim, f, eps, rope_base, dtype, max_pos, &b);
+    if (r != LB_OK) {
+      const std::string msg = g_last_error;
+      llama_stack_destroy(st);
+      return fail(r, "stack_create: layer %d: %s", l, msg.c_str());
+    }
+    st->layers.push_back(b);
+  }
+  st->d = d;
+  st->esz = dtype == LB_F32 ? 4 : 2;
+  *out = st;
+  return LB_OK;
+}
+
+llama_block* llama_stack_layer(llama_stack* st, int layer) {
+  if (!st || layer < 0 || layer >= (int)st->layers.size()) return nullptr;
+  return st->layers[layer];
+}
+
+lb_status llama_stack_set_lengths(llama_stack* st, const int32_t* lens_host, int B) {
+  if (!st) return fail(LB_ERR_INVALID_ARG, "stack_set_lengths: NULL stack");
+  for (llama_block* b : st->layers) {
+    const lb_status r = llama_block_set_lengths(b, lens_host, B);
+    if (r != LB_OK) return r;
+  }
+  return LB_OK;
+}
+
+}  // extern "C"
+
+enum StackOp { kStackPrefill, kStackExtend, kStackDecode };
+
+static lb_status stack_run(llama_stack* st, StackOp op, const void* x, void* y, int B, int T,
+                           void* const* k_caches, void* const* v_caches, int t_max,
+                           int32_t* cache_len, void* stream) {
+  const char* who = op == kStackPrefill ? "stack_prefill" : op == kStackExtend ? "stack_extend" : "stack_decode";
+  if (!st || !x || !y || !k_caches || !v_caches || !cache_len)
+    return fail(LB_ERR_INVALID_ARG, "%s: NULL argument", who);
+  if (B <= 0 || T <= 0) return fail(LB_ERR_INVALID_ARG, "%s: B and T must be positive", who);
+  if (x == y) return fail(LB_ERR_INVALID_ARG, "%s: y must not alias x", who);
+  const int n = (int)st->layers.size();
+  for (int l = 0; l < n; ++l)
+    if (!k_caches[l] || !v_caches[l])
+      return fail(LB_ERR_INVALID_ARG, "%s: NULL cache pointer for layer %d", who, l);
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t act = (size_t)B * T * st->d * st->esz;
+  if (n > 1 && act > st->act_bytes) {
+    LB_CUDA(cudaDeviceSynchronize());
+    for (int i = 0; i < 2; ++i) {
+      if (st->act[i]) LB_CUDA(cudaFree(st->act[i]));
+      st->act[i] = nullptr;
+    }
+    st->act_bytes = 0;
+    LB_CUDA(cudaMalloc(&st->act[0], act));
+    LB_CUDA(cudaMalloc(&st->act[1], act));
+    st->act_bytes = act;
+  }
+  if (n * B > st->lens_cap) {
+    LB_CUDA(cudaDeviceSynchronize());
+    if (st->lens) LB_CUDA(cudaFree(st->lens));
+    st->lens = nullptr;
+    st->lens_cap = 0;
+    LB_CUDA(cudaMalloc(&st->lens, (size_t)n * B * sizeof(int32_t)));
+    st->lens_cap = n * B;
+  }
+  // every layer starts from the caller's lengths and updates its own copy
+  for (int l = 0; l < n; ++l)
+    LB_CUDA(cudaMemcpyAsync(st->lens + (size_t)l * B, cache_len, B * sizeof(int32_t),
+                            cudaMemcpyDeviceToDevice, s));
+  const void* in = x;
+  for (int l = 0; l < n; ++l) {
+    void* out = l == n - 1 ? y : st->act[l & 1];
+    int32_t* ll = st->lens + (size_t)l * B;
+    lb_status r;
+    if (op == kStackPrefill)
+      r = llama_block_prefill(st->layers[l], in, out, B, T, k_caches[l], v_caches[l], t_max, ll, stream);
+    else if (op == kStackExtend)
+      r = llama_block_extend(st->layers[l], in, out, B, T, k_caches[l], v_caches[l], t_max, ll, stream);
+    else
+      r = llama_block_decode(st->layers[l], in, out, B, k_caches[l], v_caches[l], t_max, ll, stream);
+    if (r != LB_OK) {
+      const std::string msg = g_last_error;
+      return fail(r, "%s: layer %d: %s", who, l, msg.c_str());
+    }
+    in = out;
+  }
+  LB_CUDA(cudaMemcpyAsync(cache_len, st->lens + (size_t)(n - 1) * B, B * sizeof(int32_t),
+                          cudaMemcpyDeviceToDevice, s));
+  return LB_OK;
+}
+
+extern "C" {
+
+lb_status llama_stack_prefill(llama_stack* st, const void* x, void* y, int B, int T,
+                              void* const* k_caches, void* const* v_caches, int t_max,
+                              int32_t* cache_len, void* stream) {
+  return stack_run(st, kStackPrefill, x, y, B, T, k_caches, v_caches, t_max, cache_len, stream);
+}
+
+lb_status llama_stack_extend(llama_stack* st, const void* x, void* y, int B, int T,
+                             void* const* k_caches, void* const* v_caches, int t_max,
+                             int32_t* cache_len, void* stream) {
+  return stack_run(st, kStackExtend, x, y, B, T, k_caches, v_caches, t_max, cache_len, stream);
+}
+
+lb_status llama_stack_decode(llama_stack* st, const void* x, void* y, int B, void* const* k_caches,
+                             void* const* v_caches, int t_max, int32_t* cache_len, void* stream) {
+  return stack_run(st, kStackDecode, x, y, B, 1, k_caches, v_caches, t_max, cache_len, stream);
 }
 
 }  // extern "C"

@@ -141,14 +141,14 @@ __device__ __forceinline__ void epi_swiglu(uint32_t tb, int m, int nt, int M, in
 }
 
 // Columns of the fused projection: Q heads [0, H*dh), K heads, then V heads.
-// Each thread owns token row m = b*T + t at position t; RoPE pairs column i with
+// Each thread owns token row m = b*T + t at position pos0 + t; RoPE pairs column i with
 // i + dh/2 of the same head (rotate_half), both held by this thread.
 template <int BN>
 __device__ __forceinline__ void epi_qkv_rope(uint32_t tb, int m, int nt, int M, int N,
                                              const GemmEpi& e) {
   const int dh = e.dh, half = dh >> 1;
   const int b = m / e.T, t = m - (m / e.T) * e.T;
-  const int pos = t;
+  const int pos = e.pos0 + t;
   const bool row_ok = m < M;
   const float r = row_scale(e, m, M);
   bool pos_ok = pos < e.max_pos && pos < e.t_max;

@@ -75,7 +75,7 @@ cudaError_t launch_resid_rmsnorm(int dtype, const void* x, const float* partial,
                                  long long split_stride, void* x_out, const void* g, void* y,
                                  int rows, int d, float eps, cudaStream_t s);
 cudaError_t launch_qkv_finish(int dtype, const float* qkv, int n_split, long long split_stride,
-                              int M, int T, int H, int Hkv, int dh, const int* pos_base,
+                              int M, int T, int H, int Hkv, int dh, const int* pos_base, int pos0,
                               const float* cos_t, const float* sin_t, int max_pos, void* q_out,
                               void* k_cache, void* v_cache, int t_max, int* err, cudaStream_t s);
 cudaError_t launch_silu_mul(int dtype, const float* gu, int n_split, long long split_stride, int M,
@@ -122,6 +122,7 @@ struct GemmEpi {
   // kEpiQkvRope
   int f = 0;                    // kEpiSwiGLU: number of output columns (intermediate size)
   int T = 1, H = 0, Hkv = 0, dh = 128, t_max = 0, max_pos = 0;
+  int pos0 = 0;  // kEpiQkvRope: position of token 0 (the cache length before the call)
   void* q_out = nullptr;
   void* k_cache = nullptr;
   void* v_cache = nullptr;

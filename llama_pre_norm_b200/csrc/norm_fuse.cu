@@ -89,7 +89,7 @@ cudaError_t launch_resid_rmsnorm(int dtype, const void* x, const float* partial,
 // ---------------------------------------------------------------- QKV finish
 // qkv[s][m][n], n in [0, (H + 2 Hkv) * dh): columns of Q heads, then K, then V
 // (the fused projection). Sums the splits, rotates Q and K at position
-// pos = pos_base[b] + t (row m = b * T + t; pos_base NULL -> 0) using the
+// pos = pos_base[b] + pos0 + t (row m = b * T + t; pos_base NULL -> 0) using the
 // fp32 cos/sin table [max_pos][dh/2], and writes
 //   Q -> q_out[b][h][t][:]          ([B, H, T, dh])
 //   K -> k_cache[b][hk][pos][:]      ([B, Hkv, t_max, dh]), V likewise.
@@ -97,7 +97,8 @@ cudaError_t launch_resid_rmsnorm(int dtype, const void* x, const float* partial,
 template <typename T>
 __global__ void qkv_finish_kernel(const float* __restrict__ qkv, int n_split,
                                   long long split_stride, int M, int T_, int H, int Hkv, int dh,
-                                  const int* __restrict__ pos_base, const float* __restrict__ cos_t,
+                                  const int* __restrict__ pos_base, int pos0,
+                                  const float* __restrict__ cos_t,
                                   const float* __restrict__ sin_t, int max_pos, T* __restrict__ q_out,
                                   T* __restrict__ k_cache, T* __restrict__ v_cache, int t_max,
                                   int* err) {
@@ -113,7 +114,7 @@ __global__ void qkv_finish_kernel(const float* __restrict__ qkv, int n_split,
     const int hh = (idx / half) % heads;
     const int m = idx / ((long long)half * heads);
     const int b = m / T_, t = m % T_;
-    const int pos = (pos_base ? pos_base[b] : 0) + t;
+    const int pos = (pos_base ? pos_base[b] : 0) + pos0 + t;
     const long long c1 = (long long)hh * dh + i;
     float x1 = 0.f, x2 = 0.f;
     for (int s = 0; s < n_split; ++s) {
@@ -148,7 +149,7 @@ __global__ void qkv_finish_kernel(const float* __restrict__ qkv, int n_split,
 }
 
 cudaError_t launch_qkv_finish(int dtype, const float* qkv, int n_split, long long split_stride,
-                              int M, int T, int H, int Hkv, int dh, const int* pos_base,
+                              int M, int T, int H, int Hkv, int dh, const int* pos_base, int pos0,
                               const float* cos_t, const float* sin_t, int max_pos, void* q_out,
                               void* k_cache, void* v_cache, int t_max, int* err, cudaStream_t s) {
   const long long total = (long long)M * (H + 2 * Hkv) * (dh / 2);
@@ -157,10 +158,10 @@ cudaError_t launch_qkv_finish(int dtype, const float* qkv, int n_split, long lon
   const int blocks = (int)std::min<long long>((total + threads - 1) / threads, 148LL * 16);
   if (dtype == kF32)
     return launch_k(qkv_finish_kernel<float>, blocks, threads, 0, s, qkv, n_split, split_stride, M,
-                    T, H, Hkv, dh, pos_base, cos_t, sin_t, max_pos, (float*)q_out,
+                    T, H, Hkv, dh, pos_base, pos0, cos_t, sin_t, max_pos, (float*)q_out,
                     (float*)k_cache, (float*)v_cache, t_max, err);
   return launch_k(qkv_finish_kernel<bf16>, blocks, threads, 0, s, qkv, n_split, split_stride, M, T,
-                  H, Hkv, dh, pos_base, cos_t, sin_t, max_pos, (bf16*)q_out, (bf16*)k_cache,
+                  H, Hkv, dh, pos_base, pos0, cos_t, sin_t, max_pos, (bf16*)q_out, (bf16*)k_cache,
                   (bf16*)v_cache, t_max, err);
 }
 

@@ -285,6 +285,68 @@ def block_decode(x, W: dict, n_heads: int, n_kv_heads: int, head_dim: int,
             "k_new": k_new, "v_new": v_new}
 
 
+def block_extend(x, W: dict, n_heads: int, n_kv_heads: int, head_dim: int, eps: float,
+                 rope_base: float, k_cache, v_cache, L: int) -> dict:
+    """Append T new tokens x [B, T, d] to sequences that already hold L cached
+    (post-RoPE) keys/values each (chunked prefill). The new tokens sit at
+    positions L .. L+T-1 (mechanics page chapter 04: positions follow the cache
+    length); token i attends to the L cached keys and to new tokens 0..i.
+    Returns y [B, T, d], the new keys/values k_new, v_new [B, H_kv, T, d_h] and
+    the branch outputs."""
+    x = _f64(x)
+    kc, vc = _f64(k_cache), _f64(v_cache)
+    B, T, d = x.shape
+    H, Hkv, dh = n_heads, n_kv_heads, head_dim
+    h = rmsnorm(x, W["g_attn"], eps)
+    q = _split_heads(linear(h, W["wq"]), H, dh)
+    k = _split_heads(linear(h, W["wk"]), Hkv, dh)
+    v = _split_heads(linear(h, W["wv"]), Hkv, dh)
+    pos = (L + np.arange(T, dtype=np.float64))[None, None, :]
+    q = apply_rope(q, pos, rope_base)
+    k = apply_rope(k, pos, rope_base)
+    K_all = np.concatenate([kc[:, :, :L], k], axis=2)
+    V_all = np.concatenate([vc[:, :, :L], v], axis=2)
+    o = causal_attention(q, K_all, V_all)  # queries sit at the last T positions
+    o_flat = _merge_heads(o)
+    attn = linear(o_flat, W["wo"])
+    x1 = x + attn
+    h2 = rmsnorm(x1, W["g_mlp"], eps)
+    mlp = swiglu_mlp(h2, W["w_gate"], W["w_up"], W["w_down"])
+    return {"y": x1 + mlp, "x1": x1, "attn": attn, "mlp": mlp, "o": o_flat,
+            "k_new": k, "v_new": v}
+
+
+# --------------------------------------------------------------------------
+# A stack of blocks — the "x L blocks" of the chapter-02 diagram of [Mechanics]
+# and the 32 decoder layers of [LMDrive] §1/§5: layer l's output is layer l+1's
+# input; each layer has its own KV cache.
+# --------------------------------------------------------------------------
+def stack_prefill(X, Ws: list, n_heads: int, n_kv_heads: int, head_dim: int, eps: float,
+                  rope_base: float) -> dict:
+    """Prefill through len(Ws) layers. Returns y and the per-layer caches."""
+    h = _f64(X)
+    ks, vs = [], []
+    for W in Ws:
+        out = block_prefill(h, W, n_heads, n_kv_heads, head_dim, eps, rope_base)
+        h = out["y"]
+        ks.append(out["k"])
+        vs.append(out["v"])
+    return {"y": h, "k": ks, "v": vs}
+
+
+def stack_extend(x, Ws: list, n_heads: int, n_kv_heads: int, head_dim: int, eps: float,
+                 rope_base: float, k_caches: list, v_caches: list, L: int) -> dict:
+    """Append T tokens through every layer (each layer reads its own cache)."""
+    h = _f64(x)
+    ks, vs = [], []
+    for W, kc, vc in zip(Ws, k_caches, v_caches):
+        out = block_extend(h, W, n_heads, n_kv_heads, head_dim, eps, rope_base, kc, vc, L)
+        h = out["y"]
+        ks.append(out["k_new"])
+        vs.append(out["v_new"])
+    return {"y": h, "k_new": ks, "v_new": vs}
+
+
 # --------------------------------------------------------------------------
 # KV-cache memory accounting — [Mechanics] chapter 04, "MEMORY ACCOUNTING":
 #   bytes = L x 2 x B x T x H_kv x d_h x bytes(dtype)

@@ -26,7 +26,7 @@ def declared_functions():
 
 def test_library_exports_every_declared_function():
     names = declared_functions()
-    assert "llama_block_create" in names and "causal_attn" in names and len(names) == 20
+    assert "llama_block_create" in names and "causal_attn" in names and len(names) == 28
     for n in names:
         assert hasattr(lb.lib, n), f"{n} declared in llama_block.h but not exported"
 
@@ -71,6 +71,14 @@ def test_create_null_out_and_null_handles():
     assert lb.lib.llama_block_stage_times(None, None, 0, None) == 1
     assert lb.lib.llama_block_stage_name(None, 0) == b""
     assert lb.lib.llama_block_launch_count(None) == 0
+    assert lb.lib.llama_block_extend(None, None, None, 1, 1, None, None, 1, None, None) == 1
+    assert lb.lib.llama_stack_create(0, 256, 4, 4, 64, 688, 1e-6, 1e4, 0, 64, ctypes.byref(ctypes.c_void_p())) == 1
+    assert lb.lib.llama_stack_create(1, 256, 4, 4, 64, 688, 1e-6, 1e4, 0, 64, None) == 1
+    assert lb.lib.llama_stack_layer(None, 0) is None
+    assert lb.lib.llama_stack_prefill(None, None, None, 1, 1, None, None, 1, None, None) == 1
+    assert lb.lib.llama_stack_decode(None, None, None, 1, None, None, 1, None, None) == 1
+    assert lb.lib.llama_stack_set_lengths(None, None, 1) == 1
+    lb.lib.llama_stack_destroy(None)
     lb.lib.llama_block_destroy(None)  # no-op
 
 

@@ -375,3 +375,43 @@ def test_kv_cache_bytes_ledger():
     T, layers, batch, heads, hd = 4096, 2, 3, 8, 128
     assert ob.kv_cache_bytes(layers, batch, T, heads, hd, g["example08_dtype_bytes"]) == \
         T * layers * batch * heads * hd * 2 * 4
+
+
+# ---------------------------------------------------------------- chunked prefill / stack
+def test_extend_reduces_to_prefill_and_decode():
+    """Chunked prefill: appending T2 tokens after a prefill of T1 gives the last
+    T2 rows of a prefill of T1+T2 (causal attention only looks back); at L=0 it
+    is the prefill itself; with T=1 it is the decode step."""
+    H, Hkv, dh, d, f = 4, 2, 8, 16, 24
+    W = _tiny_weights(d, H, Hkv, dh, f, seed=80)
+    X = np.random.default_rng(81).normal(size=(2, 9, d))
+    full = ob.block_prefill(X, W, H, Hkv, dh, 1e-6, 1e4)
+    pre = ob.block_prefill(X[:, :5], W, H, Hkv, dh, 1e-6, 1e4)
+    ext = ob.block_extend(X[:, 5:], W, H, Hkv, dh, 1e-6, 1e4, pre["k"], pre["v"], 5)
+    np.testing.assert_allclose(ext["y"], full["y"][:, 5:], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ext["k_new"], full["k"][:, :, 5:], rtol=1e-12, atol=1e-13)
+    z = np.zeros((2, Hkv, 0, dh))
+    np.testing.assert_allclose(ob.block_extend(X, W, H, Hkv, dh, 1e-6, 1e4, z, z, 0)["y"], full["y"],
+                               rtol=1e-13, atol=1e-13)
+    one = ob.block_extend(X[:, 5:6], W, H, Hkv, dh, 1e-6, 1e4, pre["k"], pre["v"], 5)
+    dec = ob.block_decode(X[:, 5:6], W, H, Hkv, dh, 1e-6, 1e4, pre["k"], pre["v"], [5, 5])
+    np.testing.assert_allclose(one["y"], dec["y"], rtol=1e-13, atol=1e-13)
+
+
+def test_stack_one_layer_is_the_block_and_zero_layers_pass_through():
+    """A one-layer stack is the block; layers whose o_proj and down_proj are zero
+    leave the residual stream unchanged, whatever their attention and MLP do."""
+    H, Hkv, dh, d, f = 2, 1, 4, 8, 12
+    W = _tiny_weights(d, H, Hkv, dh, f, seed=90)
+    X = np.random.default_rng(91).normal(size=(1, 6, d))
+    one = ob.stack_prefill(X, [W], H, Hkv, dh, 1e-6, 1e4)
+    ref = ob.block_prefill(X, W, H, Hkv, dh, 1e-6, 1e4)
+    np.testing.assert_array_equal(one["y"], ref["y"])
+    Z = dict(W, wo=np.zeros_like(W["wo"]), w_down=np.zeros_like(W["w_down"]))
+    three = ob.stack_prefill(X, [Z, W, Z], H, Hkv, dh, 1e-6, 1e4)
+    np.testing.assert_allclose(three["y"], ref["y"], rtol=1e-14, atol=1e-14)
+    # and the stack extend continues every layer's cache
+    pre = ob.stack_prefill(X[:, :4], [W, W], H, Hkv, dh, 1e-6, 1e4)
+    ext = ob.stack_extend(X[:, 4:], [W, W], H, Hkv, dh, 1e-6, 1e4, pre["k"], pre["v"], 4)
+    full = ob.stack_prefill(X, [W, W], H, Hkv, dh, 1e-6, 1e4)
+    np.testing.assert_allclose(ext["y"], full["y"][:, 4:], rtol=1e-12, atol=1e-12)

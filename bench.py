@@ -121,30 +121,65 @@ def replica_throughput(units_per_rank_step: int, steps: int, world: int, slowest
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
+    """Samples SM clock, power and clock-event reasons while the timed work runs:
+    an NVML thread every 10 ms (read-only queries; the GPU is found by UUID) and,
+    beside it, the nvidia-smi query line of the profiling recipe (200 ms) written
+    to gpurun_out/clocks_gpu<i>.csv."""
+
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
         self.proc = None
-        self.path = None
+        self.samples = []  # (sm_mhz, power_w, reasons bitmask)
+        self._stop = None
+        self._thread = None
+        self.max_mhz = None
+
+    def _nvml_loop(self, handle, nv):
+        import time as _t
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(handle) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                self.samples.append((sm, pw, rs))
+            except Exception:
+                pass
+            _t.sleep(0.01)
 
     def __enter__(self):
+        import threading
+        self._stop = threading.Event()
+        try:
+            import pynvml as nv
+            import torch
+            nv.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            handle = nv.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+            self._nv = nv
+            self._thread = threading.Thread(target=self._nvml_loop, args=(handle, nv), daemon=True)
+            self._thread.start()
+        except Exception:
+            self._thread = None
         out = ROOT / "gpurun_out"
         out.mkdir(exist_ok=True)
-        self.path = out / f"clocks_gpu{self.gpu}.csv"
         try:
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+            self.fh = open(out / f"clocks_gpu{self.cuda_index}.csv", "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
-        time.sleep(0.3)
+        time.sleep(0.05)
         return self
 
     def __exit__(self, *exc):
+        if self._thread:
+            self._stop.set()
+            self._thread.join(timeout=2)
         if self.proc:
             self.proc.terminate()
             try:
@@ -154,31 +189,20 @@ class ClockSampler:
             self.fh.close()
 
     def summary(self) -> dict:
-        if not self.proc or not self.path or not self.path.exists():
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        for line in self.path.read_text().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-
-        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
-        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
-        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        load = [s for s, p in zip(sm, pw) if p is not None and p > 250] or sm
-        return {"sm_mhz": statistics.median(load) if load else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(pw) if pw else None}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no NVML samples"]}
+        nv = self._nv
+        names = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                 "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                 "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                 "hw_power_brake_slowdown": nv.nvmlClocksEventReasonHwPowerBrakeSlowdown,
+                 "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        busy = [x for x in self.samples if not (x[2] & nv.nvmlClocksEventReasonGpuIdle)] or self.samples
+        reasons = sorted({n for n, bit in names.items() for x in busy if x[2] & bit})
+        sm = sorted(x[0] for x in busy)
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": sm[0], "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "busy_samples": len(busy),
+                "power_w_max": max(x[1] for x in self.samples), "source": "NVML 10 ms + nvidia-smi 200 ms"}
 
 
 # ------------------------------------------------------------------ CPU oracle baseline

@@ -131,7 +131,8 @@ __global__ void __launch_bounds__(kDecThreads, NREP >= 4 ? 1 : 2) attn_decode_sp
 
   for (int c = 0; c < nch; ++c) {
     const int st = c % kDecStages;
-    if (!mbar_wait(&full[st], (c / kDecStages) & 1, err, 0x35)) break;
+    // warp-uniform: the lanes of a warp meet in full-mask shuffles below
+    if (!mbar_wait_warp(&full[st], (c / kDecStages) & 1, err, 0x35)) break;
     const bf16* Ks = sKV + (2 * st) * (CHUNK_BYTES / 2);
     const bf16* Vs = sKV + (2 * st + 1) * (CHUNK_BYTES / 2);
     const int rows = min(kDecChunk, nk - c * kDecChunk);

@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
     float m_ref = -INFINITY, l_run = 0.f;
     bool ok = n > 0;
     for (int j = 0; j < n && ok; ++j) {
-      if (!mbar_wait(&s_full[t], j & 1, err, 0x29)) {
+      if (!mbar_wait_warp(&s_full[t], j & 1, err, 0x29)) {
         ok = false;
         break;
       }
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
       if (j > 0 && __any_sync(0xffffffffu, move)) {
         // O_t holds PV_t(j-1) in full (S_t(j) was issued after it completed); it is
         // rescaled before this tile's P is released to the MMA.
-        if (!mbar_wait(&o_full[t], (j - 1) & 1, err, 0x2a)) {
+        if (!mbar_wait_warp(&o_full[t], (j - 1) & 1, err, 0x2a)) {
           ok = false;
           break;
         }
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    if (ok && mbar_wait(&o_full[t], (n - 1) & 1, err, 0x2b)) {
+    if (ok && mbar_wait_warp(&o_full[t], (n - 1) & 1, err, 0x2b)) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       const bool store = row0 + r < Tq;

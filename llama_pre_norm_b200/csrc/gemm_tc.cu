@@ -120,6 +120,56 @@ __device__ __forceinline__ void epi_store_resid(uint32_t tb, int m, int nt, int 
   if (e.ss_out && m < M) atomicAdd(e.ss_out + m, ssq);
 }
 
+// Residual-add epilogue with the row's residual already in registers (rres: the
+// BN columns of row m, loaded before the accumulator was ready).
+template <int BN>
+__device__ __forceinline__ void prefetch_resid(uint4 (&rres)[BN / 8], int m, int nt, int M, int N,
+                                               const GemmEpi& e) {
+  const int n0 = nt * BN;
+  if (m < M && n0 + BN <= N) {
+    const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(e.resid) +
+                                                      (long long)m * e.ldo + n0);
+#pragma unroll
+    for (int i = 0; i < BN / 8; ++i) rres[i] = src[i];
+  }
+}
+
+template <int BN>
+__device__ __forceinline__ void epi_resid_prefetched(uint32_t tb, int m, int nt, int M, int N,
+                                                     const GemmEpi& e, const uint4 (&rres)[BN / 8]) {
+  const int n0 = nt * BN;
+  // ragged tile (some row of this warp or the columns out of range): the general
+  // path. The choice is warp-uniform: tcgen05.ld is a warp-collective instruction.
+  if (!__all_sync(0xffffffffu, m < M && n0 + BN <= N)) {
+    epi_store_resid<BN>(tb, m, nt, M, N, e, true);
+    return;
+  }
+  bf16* out = reinterpret_cast<bf16*>(e.out) + (long long)m * e.ldo;
+  float ssq = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    float v[32];
+    tmem_ld32(tb + c * 32, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float r[8];
+      unpack_bf16x8(rres[c * 4 + q], r);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[q * 8 + i] += r[i];
+    }
+    if (e.ss_out) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        v[i] = round_to<bf16>(v[i]);
+        ssq += v[i] * v[i];
+      }
+    }
+    store_row32(out, n0 + c * 32, N, v);
+  }
+  if (e.ss_out && m < M) atomicAdd(e.ss_out + m, ssq);
+}
+
 // Tile columns [0,128) are gate rows 128*nt.., [128,256) the matching up rows.
 __device__ __forceinline__ void epi_swiglu(uint32_t tb, int m, int nt, int M, int f,
                                            const GemmEpi& e) {
@@ -360,7 +410,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++t) {
       const Unit w = decode_unit(u, num_m, num_n, KB, kb_per);
       const int acc = t & 1;
-      if (!mbar_wait(&tfull[acc], (t >> 1) & 1, epi.err, 5)) break;
+      if (!mbar_wait_warp(&tfull[acc], (t >> 1) & 1, epi.err, 5)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
       const int m = w.mt * kBM + row_in_tile;
@@ -529,14 +579,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int u = pair; u < units; u += npairs, ++t) {
       const int mt = u % num_m, nt = u / num_m;
       const int acc = t & 1;
-      if (!mbar_wait(&tfull[acc], (t >> 1) & 1, epi.err, 0x16)) break;
+      const int m = mt * 2 * kBM + rank * kBM + row_in_tile;
+      // With a short K loop (o_proj) the residual is fetched while the accumulator
+      // is still being computed; with a long one (down_proj) measurement showed the
+      // early loads cost more than they hide, so it is read in the epilogue.
+      const bool prefetch = EPI == kEpiResid && KB <= 64;
+      uint4 rres[EPI == kEpiResid ? BN / 8 : 1];
+      if constexpr (EPI == kEpiResid)
+        if (prefetch) prefetch_resid<BN>(rres, m, nt, M, N, epi);
+      if (!mbar_wait_warp(&tfull[acc], (t >> 1) & 1, epi.err, 0x16)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
-      const int m = mt * 2 * kBM + rank * kBM + row_in_tile;
       if constexpr (EPI == kEpiStore) {
         epi_store_resid<BN>(tb, m, nt, M, N, epi, false);
       } else if constexpr (EPI == kEpiResid) {
-        epi_store_resid<BN>(tb, m, nt, M, N, epi, true);
+        if (prefetch)
+          epi_resid_prefetched<BN>(tb, m, nt, M, N, epi, rres);
+        else
+          epi_store_resid<BN>(tb, m, nt, M, N, epi, true);
       } else if constexpr (EPI == kEpiSwiGLU) {
         epi_swiglu(tb, m, nt, M, epi.f, epi);
       } else {

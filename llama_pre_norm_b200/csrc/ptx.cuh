@@ -92,6 +92,14 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Warp-uniform form of mbar_wait for warps that go on to execute warp-collective
+// (.sync.aligned) tcgen05 instructions: every lane gets the same answer, so a
+// timeout can never leave part of the warp inside tcgen05.ld / tcgen05.st.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* err, int site) {
+  const bool ok = mbar_wait(bar, parity, err, site);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ----------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -4,7 +4,8 @@
 Headline: prefill of the LLaMA-7B-shaped block (bf16, d=4096, 32 heads, head_dim
 128, f=11008, B=1, T=2048) in tokens/s, with the fraction of dense BF16 tensor
 peak it reaches; beside it, the KV-cache decode step of the same block (B=32,
-cache 4096 -> 4224 over 128 steps) in HBM GB/s.
+cache 4096 -> 4224 over 128 steps) in HBM GB/s, with bf16 and with INT8 weight-only
+projections.
 
 One step = one prefill of the whole block (RMSNorm, fused QKV GEMM with RoPE and
 the KV-cache scatter, causal attention, o_proj + residual, RMSNorm, gate/up GEMM
@@ -83,13 +84,19 @@ def prefill_flops(cfg) -> dict:
             "total": qkv + o + gu + down + attn}
 
 
-def decode_bytes(cfg, L: int) -> int:
+def decode_bytes(cfg, L: int, int8_weights: bool = False) -> int:
     """Algorithmic HBM bytes of one decode step at cache length L (before the step):
-    every weight once, K and V of L+1 keys per (sequence, KV head), the new K/V
-    written, and the activations in and out."""
+    every weight once (bf16, or INT8 codes plus one fp32 scale per output row), K and
+    V of L+1 keys per (sequence, KV head), the new K/V written, and the activations
+    in and out."""
     es = 2
     d, f, H, Hkv, dh, B = cfg.d, cfg.f, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.B
-    weights = ((H + 2 * Hkv) * dh * d + d * H * dh + 3 * d * f + 2 * d) * es
+    n_w = (H + 2 * Hkv) * dh * d + d * H * dh + 3 * d * f
+    if int8_weights:
+        rows = (H + 2 * Hkv) * dh + d + 2 * f + d
+        weights = n_w + 4 * rows + 2 * d * es
+    else:
+        weights = (n_w + 2 * d) * es
     kv_read = 2 * B * Hkv * (L + 1) * dh * es
     kv_write = 2 * B * Hkv * dh * es
     act = 2 * B * d * es
@@ -389,6 +396,28 @@ def run_ours(args):
             attn_bytes_mean = statistics.mean(decode_attn_bytes(dcfg, L) for L in Ls)
             gbs = bytes_mean / (per_step_ms * 1e-3) / 1e9
             attn_gbs = attn_bytes_mean / (statistics.mean(attn_ms) * 1e-3) / 1e9
+            # the same steps with INT8 weight-only projections (one repetition, no stage events)
+            blk.quantize_decode_weights(True, stream)
+            reset()
+            for s in range(min(args.warmup, args.decode_steps)):
+                blk.decode(xs[s], yd, kcd, vcd, dlens)
+            blk.sync_status()
+            reset()
+            w8l0 = blk.launch_count
+            barrier()
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            for s in range(args.decode_steps):
+                blk.decode(xs[s], yd, kcd, vcd, dlens)
+            ev1.record(stream)
+            ev1.synchronize()
+            barrier()
+            blk.sync_status()
+            w8_launches = blk.launch_count - w8l0
+            blk.quantize_decode_weights(False, stream)
+            w8_step_ms = max_over_ranks(ev0.elapsed_time(ev1)) / args.decode_steps
+            w8_bytes = statistics.mean(decode_bytes(dcfg, L, int8_weights=True) for L in Ls)
+            w8_gbs = w8_bytes / (w8_step_ms * 1e-3) / 1e9
             dec = {
                 "workload": f"llama7b decode B={dcfg.B}, cache {dcfg.cache_len} -> {dcfg.cache_len + args.decode_steps}",
                 "ms_per_step": per_step_ms, "hbm_gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
@@ -397,6 +426,10 @@ def run_ours(args):
                 "attention_kernel": {"ms": statistics.mean(attn_ms), "bytes_mean": attn_bytes_mean,
                                      "achieved_gbs": attn_gbs, "frac": attn_gbs / peaks["hbm_gbs"],
                                      "traffic": NCU_TRAFFIC_BYTES["attention_decode"]},
+                "int8_weights": {"ms_per_step": w8_step_ms, "hbm_gbs": w8_gbs,
+                                 "frac_of_hbm": w8_gbs / peaks["hbm_gbs"], "bytes_per_step_mean": w8_bytes,
+                                 "tokens_per_s": dcfg.B / (w8_step_ms * 1e-3) * world,
+                                 "speedup_vs_bf16": per_step_ms / w8_step_ms, "kernel_launches": w8_launches},
             }
     clk = clocks.summary()
 
@@ -453,7 +486,8 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": {"value": replica_throughput(tokens, args.steps, world, e2e_tot), "unit": UNIT,
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": X.numel() * 2},
-        "gpu_launches": prefill_launches + (dec["kernel_launches"] if dec else 0),
+        "gpu_launches": prefill_launches + (dec["kernel_launches"] + dec["int8_weights"]["kernel_launches"]
+                                            if dec else 0),
         "gpu_launches_note": "library kernels launched in the timed prefill steps and the timed decode repetitions",
         "clocks": clk,
     }

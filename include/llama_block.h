@@ -78,6 +78,16 @@ lb_status llama_block_set_weights(llama_block* blk, const void* wq, const void* 
                                   const void* w_up, const void* w_down,
                                   const void* g_attn, const void* g_mlp, void* stream);
 
+/* Weight-only INT8 for decode ("深入解析Llama MLP模块" page §6.4: INT8 weights reduce the
+ * inference memory of the MLP; a decode step streams every weight once). enable = 1:
+ * the handle quantizes its packed projection weights per output row (s = max|w|/127,
+ * q = rint(w/s) in [-127, 127], decided in fp32) into library-owned INT8 copies, and
+ * llama_block_decode with B <= 32 then reads those (half the weight bytes), applying
+ * s in the GEMM epilogue; prefill keeps the bf16 weights. Later set_weights calls
+ * re-quantize. enable = 0 frees the copies. LB_BF16 handles only; needs weights
+ * (LB_ERR_NO_WEIGHTS) and every K dimension a multiple of 64 (LB_ERR_UNSUPPORTED). */
+lb_status llama_block_quantize_decode_weights(llama_block* blk, int enable, void* stream);
+
 /* Preallocate the workspace for up to `max_tokens` prefill rows (B*T) and
  * `max_batch` decode sequences, so that later calls allocate nothing (needed
  * before capturing calls in a CUDA graph). Optional: calls grow the workspace

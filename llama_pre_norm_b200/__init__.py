@@ -19,6 +19,7 @@ import torch
 __all__ = [
     "LB_F32", "LB_BF16", "LlamaBlockError", "lib", "lib_path", "dtype_code",
     "llama_block_create", "llama_block_set_weights", "llama_block_reserve",
+    "llama_block_quantize_decode_weights",
     "llama_block_prefill", "llama_block_extend", "llama_block_decode", "llama_block_set_lengths",
     "llama_block_kv_cache_bytes", "llama_block_sync_status", "llama_block_destroy",
     "llama_block_last_error", "llama_block_selftest_timeout", "llama_block_enable_timing",
@@ -36,7 +37,7 @@ lib_path = Path(os.environ.get("LLAMA_BLOCK_LIB", Path(__file__).resolve().paren
 if not lib_path.exists():
     raise ImportError(
         f"llama_pre_norm_b200: CUDA library {lib_path} is not built "
-        "(run `python -m llama_pre_norm_b200.build`); there is no fallback path")
+        "(run `python llama_pre_norm_b200/build.py`); there is no fallback path")
 lib = ctypes.CDLL(str(lib_path))
 
 _p, _i, _f, _sz, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_longlong
@@ -45,6 +46,7 @@ _SIGS = {
     "llama_block_create": (_i, [_i, _i, _i, _i, _i, _f, _f, _i, _i, _pp]),
     "llama_block_set_weights": (_i, [_p] * 11),
     "llama_block_reserve": (_i, [_p, _i, _i]),
+    "llama_block_quantize_decode_weights": (_i, [_p, _i, _p]),
     "llama_block_prefill": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p]),
     "llama_block_extend": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p]),
     "llama_block_decode": (_i, [_p, _p, _p, _i, _p, _p, _i, _p, _p]),
@@ -133,6 +135,11 @@ def llama_block_set_weights(h, wq, wk, wv, wo, w_gate, w_up, w_down, g_attn, g_m
                                          (w_gate, "w_gate"), (w_up, "w_up"), (w_down, "w_down"),
                                          (g_attn, "g_attn"), (g_mlp, "g_mlp"))]
     _check(lib.llama_block_set_weights(h, *ptrs, _stream(stream)), "llama_block_set_weights")
+
+
+def llama_block_quantize_decode_weights(h, enable=True, stream=None):
+    _check(lib.llama_block_quantize_decode_weights(h, 1 if enable else 0, _stream(stream)),
+           "llama_block_quantize_decode_weights")
 
 
 def llama_block_reserve(h, max_tokens, max_batch):
@@ -273,6 +280,9 @@ class LlamaBlock:
 
     def reserve(self, max_tokens, max_batch):
         llama_block_reserve(self.handle, max_tokens, max_batch)
+
+    def quantize_decode_weights(self, enable=True, stream=None):
+        llama_block_quantize_decode_weights(self.handle, enable, stream)
 
     def prefill(self, x, y, k_cache, v_cache, cache_len, stream=None):
         llama_block_prefill(self.handle, x, y, k_cache, v_cache, cache_len, stream)

@@ -1,6 +1,7 @@
 """Build the CUDA library ``libllama_block.so`` in-tree for sm_100a.
 
-Usage: ``python -m llama_pre_norm_b200.build [--force] [--verbose]``.
+Usage: ``python llama_pre_norm_b200/build.py [--force] [--verbose]`` (run as a file:
+importing the package would first load the library being built).
 
 Each ``csrc/*.cu`` is compiled to an object under ``_build/`` (in parallel,
 skipped when up to date), then linked with nvcc into

@@ -85,6 +85,19 @@ bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                     uint32_t box_rows, uint32_t box_cols) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc || (reinterpret_cast<uintptr_t>(base) & 15) || cols % 16 || box_cols % 16) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_tmap_3d_bf16(CUtensorMap* m, const void* base, uint64_t planes, uint64_t rows,
                        uint64_t cols, uint64_t plane_stride, uint32_t box_rows) {
   EncodeTiledFn enc = get_encode();
@@ -143,6 +156,11 @@ struct llama_block {
   void* ws = nullptr;
   size_t ws_bytes = 0;
   std::vector<int> lens;  // host mirror of the cache lengths
+  // INT8 decode weights (llama_block_quantize_decode_weights): codes and row scales of
+  // the packed W_qkv, W_o, W_gu, W_d
+  bool decode_int8 = false;
+  void *q8[4] = {nullptr, nullptr, nullptr, nullptr};
+  float* s8[4] = {nullptr, nullptr, nullptr, nullptr};
   // profiling: optional per-stage events, and the number of kernels launched
   bool timing = false;
   std::vector<cudaEvent_t> ev;            // 2 per stage
@@ -359,7 +377,31 @@ void llama_block_destroy(llama_block* b) {
   for (void* p : {b->w_qkv, b->w_o, b->w_gu, b->w_d, b->g1, b->g2, (void*)b->cos_t,
                   (void*)b->sin_t, (void*)b->err, b->ws})
     if (p) cudaFree(p);
+  for (int i = 0; i < 4; ++i) {
+    if (b->q8[i]) cudaFree(b->q8[i]);
+    if (b->s8[i]) cudaFree(b->s8[i]);
+  }
   delete b;
+}
+
+// Rows and columns of the four packed weight matrices (Q|K|V, o_proj, gate/up, down).
+static void packed_shapes(const llama_block* b, int rows[4], int cols[4]) {
+  rows[0] = b->n_qkv;  cols[0] = b->d;
+  rows[1] = b->d;      cols[1] = b->H * b->dh;
+  rows[2] = b->n_gu;   cols[2] = b->d;
+  rows[3] = b->d;      cols[3] = b->f;
+}
+
+static lb_status quantize_packed(llama_block* b, cudaStream_t s) {
+  int rows[4], cols[4];
+  packed_shapes(b, rows, cols);
+  void* w[4] = {b->w_qkv, b->w_o, b->w_gu, b->w_d};
+  for (int i = 0; i < 4; ++i) {
+    if (!b->q8[i]) LB_CUDA(cudaMalloc(&b->q8[i], (size_t)rows[i] * cols[i]));
+    if (!b->s8[i]) LB_CUDA(cudaMalloc(&b->s8[i], (size_t)rows[i] * sizeof(float)));
+    LB_CUDA(launch_quantize_rows_int8(w[i], b->q8[i], b->s8[i], rows[i], cols[i], s));
+  }
+  return LB_OK;
 }
 
 lb_status llama_block_set_weights(llama_block* b, const void* wq, const void* wk, const void* wv,
@@ -413,6 +455,33 @@ lb_status llama_block_set_weights(llama_block* b, const void* wq, const void* wk
     LB_CUDA(launch_scale_cols(b->w_gu, g_mlp, b->n_gu, b->d, s));
   }
   b->has_weights = true;
+  if (b->decode_int8) return quantize_packed(b, s);  // keep the INT8 copies in step
+  return LB_OK;
+}
+
+lb_status llama_block_quantize_decode_weights(llama_block* b, int enable, void* stream) {
+  if (!b) return fail(LB_ERR_INVALID_ARG, "quantize_decode_weights: NULL handle");
+  if (!enable) {
+    LB_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+    for (int i = 0; i < 4; ++i) {
+      if (b->q8[i]) LB_CUDA(cudaFree(b->q8[i]));
+      if (b->s8[i]) LB_CUDA(cudaFree(b->s8[i]));
+      b->q8[i] = nullptr;
+      b->s8[i] = nullptr;
+    }
+    b->decode_int8 = false;
+    return LB_OK;
+  }
+  if (b->dtype != kBF16)
+    return fail(LB_ERR_UNSUPPORTED, "quantize_decode_weights: INT8 decode weights need LB_BF16");
+  if (!b->has_weights) return fail(LB_ERR_NO_WEIGHTS, "quantize_decode_weights: set_weights first");
+  int rows[4], cols[4];
+  packed_shapes(b, rows, cols);
+  for (int i = 0; i < 4; ++i)
+    if (cols[i] % 64) return fail(LB_ERR_UNSUPPORTED, "quantize_decode_weights: K %% 64 != 0");
+  const lb_status st = quantize_packed(b, (cudaStream_t)stream);
+  if (st != LB_OK) return st;
+  b->decode_int8 = true;
   return LB_OK;
 }
 
@@ -559,6 +628,13 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
   b->stage_names.clear();
   if (b->dtype == kBF16) {
     const int bn = B <= 32 ? 32 : B <= 64 ? 64 : B <= 128 ? 128 : 256;
+    const bool w8 = b->decode_int8 && B <= 32;
+    // weight matrix i as the decode GEMM's 128-row operand: INT8 codes + row scales, or bf16
+    auto wgemm = [&](int i, const void* wbf, const void* act, int Mw, int Kw, int split,
+                     const GemmEpi& ep) -> cudaError_t {
+      if (w8) return launch_gemm_w8(b->q8[i], b->s8[i], act, Mw, B, Kw, split, ep, b->num_sms, s);
+      return launch_gemm_tc(wbf, act, Mw, B, Kw, bn, split, ep, b->num_sms, s);
+    };
     // gains are folded into W_qkv / W_gu: the norms here only scale by 1/RMS
     LB_STAGE("rmsnorm_attn", 1,
              launch_resid_rmsnorm(kBF16, x, nullptr, 0, 0, nullptr, nullptr, w.h, B, d, b->eps, s));
@@ -567,7 +643,7 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
     e.kind = kEpiPartialT; e.out = w.part; e.err = b->err;
     e.ldo = b->n_qkv; e.split_stride = (long long)B * b->n_qkv;
     const int s1 = decode_split((b->n_qkv + 127) / 128, d);
-    LB_STAGE("qkv_gemm", 1, launch_gemm_tc(b->w_qkv, w.h, b->n_qkv, B, d, bn, s1, e, b->num_sms, s));
+    LB_STAGE("qkv_gemm", 1, wgemm(0, b->w_qkv, w.h, b->n_qkv, d, s1, e));
     LB_STAGE("qkv_rope_append", 1,
              launch_qkv_finish(kBF16, w.part, gemm_effective_split(d, s1), e.split_stride, B, 1, H,
                                Hkv, dh, cache_len, 0, b->cos_t, b->sin_t, b->max_pos, w.q, k_cache,
@@ -578,20 +654,20 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
     const int K2 = H * dh;
     const int s2 = decode_split((d + 127) / 128, K2);
     e.ldo = d; e.split_stride = (long long)B * d;
-    LB_STAGE("o_proj_gemm", 1, launch_gemm_tc(b->w_o, w.o, d, B, K2, bn, s2, e, b->num_sms, s));
+    LB_STAGE("o_proj_gemm", 1, wgemm(1, b->w_o, w.o, d, K2, s2, e));
     LB_STAGE("resid_rmsnorm_mlp", 1,
              launch_resid_rmsnorm(kBF16, x, w.part, gemm_effective_split(K2, s2), e.split_stride,
                                   w.x1, nullptr, w.h, B, d, b->eps, s));
     // gate/up (packed rows), SiLU(g) * u
     const int s3 = decode_split((b->n_gu + 127) / 128, d);
     e.ldo = b->n_gu; e.split_stride = (long long)B * b->n_gu;
-    LB_STAGE("gate_up_gemm", 1, launch_gemm_tc(b->w_gu, w.h, b->n_gu, B, d, bn, s3, e, b->num_sms, s));
+    LB_STAGE("gate_up_gemm", 1, wgemm(2, b->w_gu, w.h, b->n_gu, d, s3, e));
     LB_STAGE("silu_mul", 1, launch_silu_mul(kBF16, w.part, gemm_effective_split(d, s3), e.split_stride,
                                             B, f, b->n_gu, 128, w.a, s));
     // down, y = X' + sum(partials); cache_len += 1
     const int s4 = decode_split((d + 127) / 128, f);
     e.ldo = d; e.split_stride = (long long)B * d;
-    LB_STAGE("down_gemm", 1, launch_gemm_tc(b->w_d, w.a, d, B, f, bn, s4, e, b->num_sms, s));
+    LB_STAGE("down_gemm", 1, wgemm(3, b->w_d, w.a, d, f, s4, e));
     LB_STAGE("resid_add_len", 1, launch_resid_add(kBF16, w.x1, w.part, gemm_effective_split(f, s4),
                                                   e.split_stride, y, (long long)B * d, cache_len, B,
                                                   1, s));

@@ -144,6 +144,16 @@ struct GemmEpi {
 cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, int BN, int n_split,
                            const GemmEpi& epi, int num_sms, cudaStream_t s);
 
+// ----------------------------------------------------------- gemm_w8.cu (INT8 weights, decode)
+// q[r][c] = rint(w[r][c] / s_r), s_r = max_c |w[r][c]| / 127 (fp32), bf16 w [rows, cols].
+cudaError_t launch_quantize_rows_int8(const void* w, void* q, float* scale, int rows, int cols,
+                                      cudaStream_t s);
+// Swap-AB decode GEMM with INT8 weights A8 [M, K] (row scales row_scale[M]) and bf16
+// tokens B [N <= 32, K]: part[split][token][row] = row_scale[row] * sum_k A8 B (kEpiPartialT
+// layout). K % 64 == 0.
+cudaError_t launch_gemm_w8(const void* A8, const float* row_scale, const void* B, int M, int N,
+                           int K, int n_split, const GemmEpi& epi, int num_sms, cudaStream_t s);
+
 // ----------------------------------------------------------- attn_tc.cu (bf16 tcgen05)
 // Causal flash attention. q [B,H,Tq,dh]; k,v [B,Hkv,k_stride,dh]; o [B,Tq,H*dh].
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o, int B, int Tq,
@@ -164,6 +174,10 @@ cudaError_t launch_attn_decode(const void* q, const void* k, const void* v, void
 // box of [box_rows, 64 cols] and 128-byte swizzle.
 bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                        uint32_t box_rows);
+// 2D uint8 tensor map over a row-major [rows, cols] byte matrix, box [box_rows,
+// box_cols], no swizzle.
+bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                     uint32_t box_rows, uint32_t box_cols);
 // 3D bf16 tensor map over [planes, rows, cols] (cols contiguous, rows `cols` apart,
 // planes `plane_stride` elements apart), box [1, box_rows, 64], 128-byte swizzle.
 // Rows >= `rows` read as zero.

@@ -348,6 +348,39 @@ def stack_extend(x, Ws: list, n_heads: int, n_kv_heads: int, head_dim: int, eps:
 
 
 # --------------------------------------------------------------------------
+# Weight-only INT8 for decode ("深入解析Llama MLP模块" §6.4 recommends INT8 weights to
+# cut inference memory; the page gives no scheme). Reading taken: symmetric,
+# per output row (per nn.Linear output feature): s = max|w| / 127, q = rint(w / s)
+# in [-127, 127], w ~ s * q. The scale and the rounding decide integers, so they
+# are taken in fp32 exactly as the GPU takes them (IEEE division, round half to
+# even); everything after that is fp64.
+# --------------------------------------------------------------------------
+def quantize_int8_rows(w):
+    """Per-row symmetric INT8 codes and fp32 scales of a weight matrix [out, in]."""
+    w32 = np.asarray(_f64(w), dtype=np.float32)
+    amax = np.max(np.abs(w32), axis=1)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    q = np.rint(w32 / safe[:, None]).astype(np.float32)
+    q = np.clip(q, -127, 127)
+    q = np.where(s[:, None] > 0, q, 0).astype(np.int8)
+    return q, s
+
+
+def dequantize_int8_rows(q, s) -> np.ndarray:
+    return np.asarray(s, dtype=np.float64)[:, None] * np.asarray(q, dtype=np.float64)
+
+
+def int8_decode_weights(W: dict) -> dict:
+    """The block weights as the INT8 decode path sees them: every projection
+    replaced by its dequantized INT8 form (RMSNorm gains unchanged)."""
+    out = dict(W)
+    for k in ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down"):
+        out[k] = dequantize_int8_rows(*quantize_int8_rows(W[k]))
+    return out
+
+
+# --------------------------------------------------------------------------
 # KV-cache memory accounting — [Mechanics] chapter 04, "MEMORY ACCOUNTING":
 #   bytes = L x 2 x B x T x H_kv x d_h x bytes(dtype)
 # --------------------------------------------------------------------------

@@ -415,3 +415,33 @@ def test_stack_one_layer_is_the_block_and_zero_layers_pass_through():
     ext = ob.stack_extend(X[:, 4:], [W, W], H, Hkv, dh, 1e-6, 1e4, pre["k"], pre["v"], 4)
     full = ob.stack_prefill(X, [W, W], H, Hkv, dh, 1e-6, 1e4)
     np.testing.assert_allclose(ext["y"], full["y"][:, 4:], rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- INT8 decode weights
+def test_int8_row_quantization_properties():
+    """Per-row symmetric INT8: codes in [-127, 127], each non-zero row reaches
+    |q| = 127 at its absmax, the reconstruction error is at most half a step,
+    weights that are exact multiples of the step are reproduced exactly, and a
+    zero row stays zero."""
+    rng = np.random.default_rng(100)
+    w = rng.normal(size=(16, 64)).astype(np.float32) * 0.02
+    w[3] = 0.0
+    step = np.float32(0.125)
+    w[5] = step * rng.integers(-127, 128, size=64).astype(np.float32)
+    w[5, 0] = 127 * step
+    q, s = ob.quantize_int8_rows(w)
+    assert q.dtype == np.int8 and s.dtype == np.float32
+    assert q.min() >= -127 and q.max() <= 127
+    for r in range(16):
+        if r == 3:
+            assert s[r] == 0 and np.all(q[r] == 0)
+            continue
+        assert np.max(np.abs(q[r].astype(int))) == 127
+        err = np.abs(ob.dequantize_int8_rows(q[r:r + 1], s[r:r + 1])[0] - w[r].astype(np.float64))
+        assert np.all(err <= 0.5 * float(s[r]) * (1 + 1e-6))
+    np.testing.assert_array_equal(ob.dequantize_int8_rows(q[5:6], s[5:6])[0], w[5].astype(np.float64))
+    # the decode block on INT8 weights is the block on the dequantized weights
+    W = _tiny_weights(d=8, H=2, Hkv=1, dh=4, f=12, seed=101)
+    Wq = ob.int8_decode_weights(W)
+    assert set(Wq) == set(W) and np.array_equal(Wq["g_attn"], W["g_attn"])
+    assert not np.array_equal(Wq["wq"], W["wq"])

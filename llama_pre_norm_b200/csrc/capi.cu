@@ -85,19 +85,6 @@ bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                     uint32_t box_rows, uint32_t box_cols) {
-  EncodeTiledFn enc = get_encode();
-  if (!enc || (reinterpret_cast<uintptr_t>(base) & 15) || cols % 16 || box_cols % 16) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 bool make_tmap_3d_bf16(CUtensorMap* m, const void* base, uint64_t planes, uint64_t rows,
                        uint64_t cols, uint64_t plane_stride, uint32_t box_rows) {
   EncodeTiledFn enc = get_encode();
@@ -207,11 +194,49 @@ struct DecodeWs {
   float* attn_part;
 };
 
-static int decode_split(int tiles, int K) {
+// Split-K factor of a decode GEMM (m_tiles x n_tiles output tiles, K deep, tile_bytes
+// streamed per 64-deep K block of a tile): the split whose busiest SM streams the
+// fewest bytes -- whole waves of equal units over the SMs, a fixed cost per unit, and
+// the fp32 partials (written, then read by the reduction) spread over all SMs.
+static int decode_split(int m_tiles, int n_tiles, int bn, int K, int tile_bytes, int num_sms) {
   const int KB = (K + 63) / 64;
-  int s = (296 + tiles - 1) / tiles;
-  s = std::max(1, std::min(s, std::max(1, KB / 4)));
-  return s;
+  const long long tiles = (long long)m_tiles * n_tiles;
+  double best = 0;
+  int best_s = 1;
+  for (int sp = 1; sp <= std::min(KB, 64); ++sp) {
+    const int per = (KB + sp - 1) / sp;
+    if ((KB + per - 1) / per != sp) continue;  // the same units as a smaller split
+    const long long units = tiles * sp;
+    const long long waves = (units + num_sms - 1) / num_sms;
+    const double cost = (double)waves * ((double)per * tile_bytes + 4096.0) +
+                        (double)units * 128.0 * bn * 4 * 2 / num_sms;
+    if (sp == 1 || cost < best * 0.999) {
+      best = cost;
+      best_s = sp;
+    }
+  }
+  return best_s;
+}
+
+// Tile width and split of the four decode GEMMs (QKV, o_proj, gate/up, down) for a
+// batch of B tokens, with the INT8 weights when w8 (used for B <= 32 only).
+struct DecodePlan {
+  int bn;
+  bool w8;
+  int split[4];
+};
+
+static DecodePlan decode_plan(const llama_block* b, int B, bool w8) {
+  DecodePlan p;
+  p.bn = B <= 32 ? 32 : B <= 64 ? 64 : B <= 128 ? 128 : 256;
+  p.w8 = w8 && B <= 32;
+  const int n_tiles = (B + p.bn - 1) / p.bn;
+  const int tile_bytes = (p.w8 ? 128 * 64 : 128 * 64 * 2) + p.bn * 64 * 2;
+  const int M[4] = {b->n_qkv, b->d, b->n_gu, b->d};
+  const int K[4] = {b->d, b->H * b->dh, b->d, b->f};
+  for (int i = 0; i < 4; ++i)
+    p.split[i] = decode_split((M[i] + 127) / 128, n_tiles, p.bn, K[i], tile_bytes, b->num_sms);
+  return p;
 }
 
 static PrefillWs carve_prefill(const llama_block* b, void* base, int M, size_t* total) {
@@ -245,12 +270,14 @@ static DecodeWs carve_decode(const llama_block* b, void* base, int B, int t_max,
   w.a = c.take((size_t)B * b->f_pad * b->esz);
   size_t part = 0;
   if (b->dtype == kBF16) {
-    const int s1 = decode_split((b->n_qkv + 127) / 128, b->d);
-    const int s2 = decode_split((b->d + 127) / 128, b->H * b->dh);
-    const int s3 = decode_split((b->n_gu + 127) / 128, b->d);
-    const int s4 = decode_split((b->d + 127) / 128, b->f);
-    part = std::max({(size_t)s1 * B * b->n_qkv, (size_t)s2 * B * b->d, (size_t)s3 * B * b->n_gu,
-                     (size_t)s4 * B * b->d});
+    // room for the partials of every batch size up to B, bf16 or INT8 weights, so that
+    // a workspace reserved for B is never regrown by a smaller decode
+    const size_t M[4] = {(size_t)b->n_qkv, (size_t)b->d, (size_t)b->n_gu, (size_t)b->d};
+    for (int bb = 1; bb <= B; ++bb)
+      for (int w8 = 0; w8 < 2; ++w8) {
+        const DecodePlan p = decode_plan(b, bb, w8 != 0);
+        for (int i = 0; i < 4; ++i) part = std::max(part, (size_t)p.split[i] * bb * M[i]);
+      }
   } else {
     part = std::max((size_t)B * b->n_qkv, (size_t)B * b->n_gu);
   }
@@ -397,8 +424,10 @@ static lb_status quantize_packed(llama_block* b, cudaStream_t s) {
   packed_shapes(b, rows, cols);
   void* w[4] = {b->w_qkv, b->w_o, b->w_gu, b->w_d};
   for (int i = 0; i < 4; ++i) {
-    if (!b->q8[i]) LB_CUDA(cudaMalloc(&b->q8[i], (size_t)rows[i] * cols[i]));
+    const size_t qbytes = w8_blocked_bytes(rows[i], cols[i]);
+    if (!b->q8[i]) LB_CUDA(cudaMalloc(&b->q8[i], qbytes));
     if (!b->s8[i]) LB_CUDA(cudaMalloc(&b->s8[i], (size_t)rows[i] * sizeof(float)));
+    LB_CUDA(cudaMemsetAsync(b->q8[i], 0, qbytes, s));  // the padding rows of the last tile
     LB_CUDA(launch_quantize_rows_int8(w[i], b->q8[i], b->s8[i], rows[i], cols[i], s));
   }
   return LB_OK;
@@ -627,8 +656,9 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
 
   b->stage_names.clear();
   if (b->dtype == kBF16) {
-    const int bn = B <= 32 ? 32 : B <= 64 ? 64 : B <= 128 ? 128 : 256;
-    const bool w8 = b->decode_int8 && B <= 32;
+    const DecodePlan plan = decode_plan(b, B, b->decode_int8);
+    const int bn = plan.bn;
+    const bool w8 = plan.w8;
     // weight matrix i as the decode GEMM's 128-row operand: INT8 codes + row scales, or bf16
     auto wgemm = [&](int i, const void* wbf, const void* act, int Mw, int Kw, int split,
                      const GemmEpi& ep) -> cudaError_t {
@@ -642,7 +672,7 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
     GemmEpi e;
     e.kind = kEpiPartialT; e.out = w.part; e.err = b->err;
     e.ldo = b->n_qkv; e.split_stride = (long long)B * b->n_qkv;
-    const int s1 = decode_split((b->n_qkv + 127) / 128, d);
+    const int s1 = plan.split[0];
     LB_STAGE("qkv_gemm", 1, wgemm(0, b->w_qkv, w.h, b->n_qkv, d, s1, e));
     LB_STAGE("qkv_rope_append", 1,
              launch_qkv_finish(kBF16, w.part, gemm_effective_split(d, s1), e.split_stride, B, 1, H,
@@ -652,20 +682,20 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
                                                 dh, t_max, cache_len, b->err, s));
     // o_proj, then X' = X + sum(partials) and h2 = RMSNorm(X') in one kernel
     const int K2 = H * dh;
-    const int s2 = decode_split((d + 127) / 128, K2);
+    const int s2 = plan.split[1];
     e.ldo = d; e.split_stride = (long long)B * d;
     LB_STAGE("o_proj_gemm", 1, wgemm(1, b->w_o, w.o, d, K2, s2, e));
     LB_STAGE("resid_rmsnorm_mlp", 1,
              launch_resid_rmsnorm(kBF16, x, w.part, gemm_effective_split(K2, s2), e.split_stride,
                                   w.x1, nullptr, w.h, B, d, b->eps, s));
     // gate/up (packed rows), SiLU(g) * u
-    const int s3 = decode_split((b->n_gu + 127) / 128, d);
+    const int s3 = plan.split[2];
     e.ldo = b->n_gu; e.split_stride = (long long)B * b->n_gu;
     LB_STAGE("gate_up_gemm", 1, wgemm(2, b->w_gu, w.h, b->n_gu, d, s3, e));
     LB_STAGE("silu_mul", 1, launch_silu_mul(kBF16, w.part, gemm_effective_split(d, s3), e.split_stride,
                                             B, f, b->n_gu, 128, w.a, s));
     // down, y = X' + sum(partials); cache_len += 1
-    const int s4 = decode_split((d + 127) / 128, f);
+    const int s4 = plan.split[3];
     e.ldo = d; e.split_stride = (long long)B * d;
     LB_STAGE("down_gemm", 1, wgemm(3, b->w_d, w.a, d, f, s4, e));
     LB_STAGE("resid_add_len", 1, launch_resid_add(kBF16, w.x1, w.part, gemm_effective_split(f, s4),

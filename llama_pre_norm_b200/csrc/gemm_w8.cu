@@ -8,10 +8,12 @@
 //
 // The GEMM is the swap-AB decode GEMM of gemm_tc.cu (weights are the 128-row
 // operand, the B <= 32 tokens the N side, split-K partials) with one more stage:
-//   warp 0      TMA: the INT8 weight tile (128 x 64 bytes) and the bf16 token tile
-//   warps 6..9  convert the INT8 tile to bf16 (exact: |q| <= 127) into the MMA's
-//               128-byte-swizzled K-major layout, one weight row per thread
-//   warp 1      tcgen05.mma (M=128, N=32) on the converted tile
+//   warp 0      loads: the INT8 weight tile (128 x 64 bytes, one contiguous bulk copy
+//               from the tile-blocked layout) and the bf16 token tile (TMA), a
+//               16-deep ring
+//   warps 6..13 widen the INT8 tile to bf16 (exact: |q| <= 127) straight into TMEM
+//               (tcgen05.st), half a weight row per thread, a 4-deep ring of tiles
+//   warp 1      tcgen05.mma (M=128, N=32) with the converted tile as the TMEM A operand
 //   warps 2..5  epilogue: partial[split][token][n] = s_n * acc
 #include "common.cuh"
 #include "internal.h"
@@ -19,17 +21,17 @@
 
 namespace lb {
 
-constexpr int kW8Threads = 320;
-
 // ---------------------------------------------------------------- quantization
 // One CTA per row: amax in fp32, s = amax / 127 (IEEE division), q = rint(w / s).
+// Codes are stored tile-blocked (w8_blocked_offset); rows of the last tile past
+// `rows` are never written, so the caller zeroes the buffer first.
 __global__ void __launch_bounds__(256) quantize_rows_int8_kernel(const bf16* __restrict__ w,
                                                                  int8_t* __restrict__ q,
                                                                  float* __restrict__ scale, int cols) {
   __shared__ float red[32];
   pdl_wait();
-  const long long row = blockIdx.x;
-  const bf16* src = w + row * cols;
+  const int row = blockIdx.x;
+  const bf16* src = w + (long long)row * cols;
   float amax = 0.f;
   for (int c = threadIdx.x; c < cols; c += blockDim.x) amax = fmaxf(amax, fabsf(__bfloat162float(src[c])));
   amax = block_max(amax, red);
@@ -38,7 +40,7 @@ __global__ void __launch_bounds__(256) quantize_rows_int8_kernel(const bf16* __r
   for (int c = threadIdx.x; c < cols; c += blockDim.x) {
     float v = 0.f;
     if (s > 0.f) v = fminf(fmaxf(rintf(__bfloat162float(src[c]) / s), -127.f), 127.f);
-    q[row * cols + c] = (int8_t)(int)v;
+    q[w8_blocked_offset(row, c, cols)] = (int8_t)(int)v;
   }
 }
 
@@ -50,45 +52,87 @@ cudaError_t launch_quantize_rows_int8(const void* w, void* q, float* scale, int 
 }
 
 // ---------------------------------------------------------------- GEMM
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Four INT8 codes (bytes of u, element j in byte j) to four bf16 (two pairs, element
+// order kept). Each biased byte q + 128 becomes the low byte of the fp32 pattern
+// 0x4B0000xx = 2^23 + q + 128; subtracting 2^23 + 128 leaves q exactly, and since
+// |q| <= 127 fits bf16's significand the bf16 is the fp32's upper half, taken by a
+// byte permute. All ALU/FMA-pipe work, no int-to-float conversion instructions.
+__device__ __forceinline__ void i8x4_to_bf16x4(uint32_t u, uint32_t& lo, uint32_t& hi) {
+  const uint32_t x = u ^ 0x80808080u;
+  constexpr float kMagic = 8388736.0f;  // 2^23 + 128
+  const float f0 = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7440)) - kMagic;
+  const float f1 = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7441)) - kMagic;
+  const float f2 = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7442)) - kMagic;
+  const float f3 = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7443)) - kMagic;
+  lo = __byte_perm(__float_as_uint(f0), __float_as_uint(f1), 0x7632);
+  hi = __byte_perm(__float_as_uint(f2), __float_as_uint(f3), 0x7632);
+}
+
+constexpr int kW8ConvWarps = 8;
+constexpr int kW8Threads = (6 + kW8ConvWarps) * 32;
+
 template <int BN>
 struct W8Cfg {
-  static constexpr int STAGES = 6;
-  static constexpr int RAW_BYTES = 128 * 64;      // INT8 weight tile
-  static constexpr int B_BYTES = BN * 64 * 2;     // bf16 token tile
-  static constexpr int CVT_BYTES = 128 * 64 * 2;  // converted bf16 weight tile
-  static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
-  static constexpr int SMEM = STAGES * (RAW_BYTES + B_BYTES + CVT_BYTES) + 256 + 1024;
+  static constexpr int STAGES = 16;           // load ring: INT8 tile + token tile
+  static constexpr int A_STAGES = 4;          // converted bf16 tiles in TMEM, 32 columns each
+  static constexpr int RAW_BYTES = 128 * 64;  // INT8 weight tile
+  static constexpr int B_BYTES = BN * 64 * 2; // bf16 token tile
+  static constexpr int A_COL0 = 2 * BN;       // TMEM: two accumulators, then the A stages
+  static constexpr int TMEM_USED = 2 * BN + A_STAGES * 32;
+  static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
+                                   : TMEM_USED <= 256 ? 256 : 512;
+  static constexpr int SMEM = STAGES * (RAW_BYTES + B_BYTES) + 512 + 1024;
 };
 
 template <int BN>
 __global__ void __launch_bounds__(kW8Threads, 1)
-    gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA8, const __grid_constant__ CUtensorMap tmB,
+    gemm_w8_kernel(const uint8_t* __restrict__ A8, const __grid_constant__ CUtensorMap tmB,
                    const float* __restrict__ row_scale, int M, int N, int K, int kb_per, int n_split,
                    GemmEpi epi) {
   using C = W8Cfg<BN>;
+  constexpr int RS = C::STAGES, AS = C::A_STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sCvt = smem;                                   // STAGES x 16 KB (1024-aligned)
-  uint8_t* sB = sCvt + C::STAGES * C::CVT_BYTES;          // STAGES x BN*128 B
-  uint8_t* sRaw = sB + C::STAGES * C::B_BYTES;            // STAGES x 8 KB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + C::STAGES * C::RAW_BYTES);
-  uint64_t* full = bars;                      // TMA landed (raw + B)
-  uint64_t* empty = bars + C::STAGES;         // raw converted and B consumed
-  uint64_t* cvt_full = bars + 2 * C::STAGES;  // converted tile ready
-  uint64_t* cvt_empty = bars + 3 * C::STAGES; // converted tile consumed by the MMA
-  uint64_t* tfull = bars + 4 * C::STAGES;
+  uint8_t* sB = smem;                           // RS x BN*128 B, 1024-aligned (128-byte swizzle)
+  uint8_t* sRaw = sB + RS * C::B_BYTES;         // RS x 8 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + RS * C::RAW_BYTES);
+  uint64_t* full = bars;                // INT8 + token tile landed
+  uint64_t* empty = bars + RS;          // INT8 tile read by the converters, token tile by the MMA
+  uint64_t* a_full = bars + 2 * RS;     // converted tile in TMEM
+  uint64_t* a_empty = a_full + AS;      // converted tile consumed by the MMA
+  uint64_t* tfull = a_empty + AS;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < RS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 5);  // one MMA commit + four converter warps
-      mbar_init(&cvt_full[s], 4);
-      mbar_init(&cvt_empty[s], 1);
+      mbar_init(&empty[s], 1 + kW8ConvWarps);  // one MMA commit + every converter warp
+    }
+    for (int s = 0; s < AS; ++s) {
+      mbar_init(&a_full[s], kW8ConvWarps);
+      mbar_init(&a_empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
@@ -96,7 +140,6 @@ __global__ void __launch_bounds__(kW8Threads, 1)
     }
     mbar_init(drain, 1);
     fence_mbar_init();
-    prefetch_tmap(&tmA8);
     prefetch_tmap(&tmB);
   }
   if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -121,7 +164,7 @@ __global__ void __launch_bounds__(kW8Threads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer
+      // ---------------- loads
       uint32_t stage = 0, phase = 0;
       long long issued = 0;
       bool ok = true;
@@ -134,25 +177,27 @@ __global__ void __launch_bounds__(kW8Threads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[stage], C::RAW_BYTES + C::B_BYTES);
-          tma_load_2d(sRaw + stage * C::RAW_BYTES, &tmA8, &full[stage], kb * 64, mt * 128);
+          // one contiguous 8 KB tile of the blocked layout
+          bulk_load(sRaw + stage * C::RAW_BYTES, A8 + ((long long)mt * KB + kb) * C::RAW_BYTES,
+                    C::RAW_BYTES, &full[stage]);
           tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * 64, nt * BN);
           ++issued;
-          if (++stage == C::STAGES) {
+          if (++stage == RS) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
       pdl_trigger();
-      const long long first = issued > C::STAGES ? issued - C::STAGES : 0;
+      const long long first = issued > RS ? issued - RS : 0;
       for (long long i = first; i < issued; ++i)
-        mbar_wait(&empty[i % C::STAGES], (uint32_t)((i / C::STAGES) & 1), epi.err, 0x42);
+        mbar_wait(&empty[i % RS], (uint32_t)((i / RS) & 1), epi.err, 0x42);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer
+      // ---------------- MMA issuer: A (the converted weights) from TMEM, B from smem
       constexpr uint32_t idesc = umma_idesc_bf16(128, BN, 0, 0);
-      uint32_t stage = 0, phase = 0;
+      uint32_t rs = 0, rphase = 0, as = 0, aphase = 0;
       int t = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++t) {
@@ -163,23 +208,27 @@ __global__ void __launch_bounds__(kW8Threads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, epi.err, 0x44) ||
-              !mbar_wait(&cvt_full[stage], phase, epi.err, 0x45)) {
+          if (!mbar_wait(&full[rs], rphase, epi.err, 0x44) ||
+              !mbar_wait(&a_full[as], aphase, epi.err, 0x45)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sCvt + stage * C::CVT_BYTES);
-          const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
+          const uint32_t a_tmem = tmem_base + C::A_COL0 + as * 32;
+          const uint32_t b0 = smem_u32(sB + rs * C::B_BYTES);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(d_tmem, umma_desc_sw128(a0 + k * 32, 16, 1024),
-                      umma_desc_sw128(b0 + k * 32, 16, 1024), idesc, (kb > kb0 || k > 0) ? 1u : 0u);
-          umma_commit(&empty[stage]);
-          umma_commit(&cvt_empty[stage]);
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1;
+          for (int k = 0; k < 4; ++k)  // K = 16 per MMA: 8 columns of bf16 pairs
+            umma_bf16_tmem_a(d_tmem, a_tmem + k * 8, umma_desc_sw128(b0 + k * 32, 16, 1024), idesc,
+                             (kb > kb0 || k > 0) ? 1u : 0u);
+          umma_commit(&empty[rs]);
+          umma_commit(&a_empty[as]);
+          if (++rs == RS) {
+            rs = 0;
+            rphase ^= 1;
+          }
+          if (++as == AS) {
+            as = 0;
+            aphase ^= 1;
           }
         }
         if (!ok) break;
@@ -189,59 +238,58 @@ __global__ void __launch_bounds__(kW8Threads, 1)
       mbar_wait(drain, 0, epi.err, 0x46);
     }
   } else if (warp >= 6) {
-    // ---------------- INT8 -> bf16 converters: thread r converts weight row r
-    const int r = threadIdx.x - 6 * 32;
-    // Order of the four 16-byte reads of a row. A 16-byte access is served per 8
-    // threads (rows r0..r0+7): reads land on 16-byte bank group 4*(r&1) + i, writes of
-    // output chunk c = 2i + h on group c ^ (r&7). Taking i = g(r>>1 & 3) ^ ii with g
-    // multiplication by a generator of GF(4) ({0,1,2,3} -> {0,2,3,1}) makes both g(x)
-    // and g(x) ^ x permutations, so each 8-thread phase hits 8 distinct groups on
-    // both the read and the write side.
-    const int rot = (0x78 >> (2 * ((r >> 1) & 3))) & 3;
-    uint32_t stage = 0, phase = 0;
+    // ---------------- INT8 -> bf16 converters. A warp may only reach the TMEM lanes
+    // 32 * (warp % 4) ..+31, so lane l of converter warp w handles weight row
+    // 32 * (w % 4) + l, K half (w - 6) / 4 of the 64-deep block: 32 codes read from
+    // shared memory, widened, stored as 16 columns of bf16 pairs.
+    const int quarter = warp & 3, half = (warp - 6) >> 2;
+    const int r = quarter * 32 + lane;
+    // The tile is stored [half][row][32 bytes]; a 16-byte access is served per 8
+    // threads (rows r0..r0+7), on 16-byte bank group 2r + chunk (mod 8): rows with
+    // bit 2 set read their second chunk first, so each phase hits 8 distinct groups.
+    const int first = (r >> 2) & 1;
+    const uint32_t raw0 = smem_u32(sRaw) + half * 4096 + r * 32;
+    const uint32_t lane_addr = ((uint32_t)(quarter * 32) << 16) + C::A_COL0 + half * 16;
+    uint32_t rs = 0, rphase = 0, as = 0, aphase = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       int mt, nt, sp, kb0, kb1;
       decode(u, mt, nt, sp, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait_warp(&full[stage], phase, epi.err, 0x47) ||
-            !mbar_wait_warp(&cvt_empty[stage], phase ^ 1, epi.err, 0x48)) {
+        if (!mbar_wait_warp(&full[rs], rphase, epi.err, 0x47) ||
+            !mbar_wait_warp(&a_empty[as], aphase ^ 1, epi.err, 0x48)) {
           ok = false;
           break;
         }
-        const uint8_t* src = sRaw + stage * C::RAW_BYTES + r * 64;
-        uint8_t* dst = sCvt + stage * C::CVT_BYTES + r * 128;
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-          const int i = ii ^ rot;  // 16 int8 = bf16 chunks 2i and 2i+1
-          const uint4 raw = *reinterpret_cast<const uint4*>(src + i * 16);
-          const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
-          uint32_t pk[8];
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            // little-endian: byte j of the word is element 4w + j; sign-extend each
-            const uint32_t u = wds[w];
-            const float f0 = (float)((int32_t)(u << 24) >> 24), f1 = (float)((int32_t)(u << 16) >> 24);
-            const float f2 = (float)((int32_t)(u << 8) >> 24), f3 = (float)((int32_t)u >> 24);
-            pk[2 * w] = pack_bf16x2(f0, f1);
-            pk[2 * w + 1] = pack_bf16x2(f2, f3);
-          }
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int c = 2 * i + h;  // 16-byte chunk of the 128-byte row
-            *reinterpret_cast<uint4*>(dst + ((c ^ (r & 7)) << 4)) =
-                make_uint4(pk[4 * h], pk[4 * h + 1], pk[4 * h + 2], pk[4 * h + 3]);
-          }
-        }
-        fence_proxy_async_smem();  // generic-proxy writes -> tensor core reads
+        tc_fence_after();
+        const uint32_t src = raw0 + rs * C::RAW_BYTES;
+        const uint4 c0 = lds128(src + first * 16);
+        const uint4 c1 = lds128(src + (first ^ 1) * 16);
+        const uint4 lo = first ? c1 : c0, hi = first ? c0 : c1;  // K 0..15, K 16..31 of the half
+        uint32_t p[16];
+        i8x4_to_bf16x4(lo.x, p[0], p[1]);
+        i8x4_to_bf16x4(lo.y, p[2], p[3]);
+        i8x4_to_bf16x4(lo.z, p[4], p[5]);
+        i8x4_to_bf16x4(lo.w, p[6], p[7]);
+        i8x4_to_bf16x4(hi.x, p[8], p[9]);
+        i8x4_to_bf16x4(hi.y, p[10], p[11]);
+        i8x4_to_bf16x4(hi.z, p[12], p[13]);
+        i8x4_to_bf16x4(hi.w, p[14], p[15]);
+        tmem_st16(tmem_base + lane_addr + as * 32, p);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&cvt_full[stage]);
-          mbar_arrive(&empty[stage]);
+          mbar_arrive(&a_full[as]);
+          mbar_arrive(&empty[rs]);
         }
-        if (++stage == C::STAGES) {
-          stage = 0;
-          phase ^= 1;
+        if (++rs == RS) {
+          rs = 0;
+          rphase ^= 1;
+        }
+        if (++as == AS) {
+          as = 0;
+          aphase ^= 1;
         }
       }
     }
@@ -293,8 +341,8 @@ cudaError_t launch_gemm_w8(const void* A8, const float* row_scale, const void* B
   if (N > 32 || K % 64 != 0) return cudaErrorInvalidValue;
   constexpr int BN = 32;
   using C = W8Cfg<BN>;
-  CUtensorMap ta, tb;
-  if (!make_tmap_2d_u8(&ta, A8, (uint64_t)M, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
+  CUtensorMap tb;
+  if (reinterpret_cast<uintptr_t>(A8) & 15) return cudaErrorInvalidValue;
   if (!make_tmap_2d_bf16(&tb, B, (uint64_t)N, (uint64_t)K, BN)) return cudaErrorInvalidValue;
   const int KB = K / 64;
   n_split = gemm_effective_split(K, n_split);
@@ -308,8 +356,8 @@ cudaError_t launch_gemm_w8(const void* A8, const float* row_scale, const void* B
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_k(kern, grid, kW8Threads, C::SMEM, s, ta, tb, row_scale, M, N, K, kb_per, n_split,
-                  epi);
+  return launch_k(kern, grid, kW8Threads, C::SMEM, s, (const uint8_t*)A8, tb, row_scale, M, N, K,
+                  kb_per, n_split, epi);
 }
 
 }  // namespace lb

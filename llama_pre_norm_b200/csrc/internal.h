@@ -145,12 +145,21 @@ cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, in
                            const GemmEpi& epi, int num_sms, cudaStream_t s);
 
 // ----------------------------------------------------------- gemm_w8.cu (INT8 weights, decode)
-// q[r][c] = rint(w[r][c] / s_r), s_r = max_c |w[r][c]| / 127 (fp32), bf16 w [rows, cols].
+// INT8 codes are stored tile-blocked so that a decode GEMM streams each 128 x 64 tile
+// as one contiguous 8 KB run, [ceil(rows/128)][cols/64] tiles (cols % 64 == 0, rows
+// padded to a multiple of 128 with zero codes), each tile [2 halves of K][128 rows][32].
+__host__ __device__ inline long long w8_blocked_offset(int row, int col, int cols) {
+  return ((long long)(row >> 7) * (cols >> 6) + (col >> 6)) * 8192 + ((col >> 5) & 1) * 4096 +
+         (row & 127) * 32 + (col & 31);
+}
+inline size_t w8_blocked_bytes(int rows, int cols) { return (size_t)((rows + 127) / 128) * 128 * cols; }
+// q = rint(w / s_r), s_r = max_c |w[r][c]| / 127 (fp32), bf16 w [rows, cols] -> blocked q
+// (zeroed beforehand by the caller), scale[rows].
 cudaError_t launch_quantize_rows_int8(const void* w, void* q, float* scale, int rows, int cols,
                                       cudaStream_t s);
-// Swap-AB decode GEMM with INT8 weights A8 [M, K] (row scales row_scale[M]) and bf16
-// tokens B [N <= 32, K]: part[split][token][row] = row_scale[row] * sum_k A8 B (kEpiPartialT
-// layout). K % 64 == 0.
+// Swap-AB decode GEMM with blocked INT8 weights A8 (M rows, row scales row_scale[M]) and
+// bf16 tokens B [N <= 32, K]: part[split][token][row] = row_scale[row] * sum_k A8 B
+// (kEpiPartialT layout). K % 64 == 0.
 cudaError_t launch_gemm_w8(const void* A8, const float* row_scale, const void* B, int M, int N,
                            int K, int n_split, const GemmEpi& epi, int num_sms, cudaStream_t s);
 
@@ -174,10 +183,6 @@ cudaError_t launch_attn_decode(const void* q, const void* k, const void* v, void
 // box of [box_rows, 64 cols] and 128-byte swizzle.
 bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                        uint32_t box_rows);
-// 2D uint8 tensor map over a row-major [rows, cols] byte matrix, box [box_rows,
-// box_cols], no swizzle.
-bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                     uint32_t box_rows, uint32_t box_cols);
 // 3D bf16 tensor map over [planes, rows, cols] (cols contiguous, rows `cols` apart,
 // planes `plane_stride` elements apart), box [1, box_rows, 64], 128-byte swizzle.
 // Rows >= `rows` read as zero.

@@ -7,8 +7,13 @@ INT8 rounding noise alone moves a decode row by about 1e-2 of its max-norm, half
 the bf16 tolerance, so agreement with the INT8 oracle does not show that the INT8
 weights were used. The per-GEMM cases therefore plant one outlier per row in one
 weight group (each row's outlier in a different column), which makes the INT8 and
-the bf16 results of the oracle differ by several tolerances; the GPU must match
-the INT8 one and be far from the bf16 one.
+the bf16 results of the oracle differ by two tolerances or more; the GPU must match
+the INT8 one and miss the bf16 one. A further case makes both paths compute the same
+products exactly and asks for bit equality.
+
+The projections have std 0.15 so that the branches, not the residual, dominate y;
+W_q and W_k keep std 0.02, since larger q and k make the softmax so sharp that bf16
+storage of q and k alone moves y by more than a tolerance.
 """
 
 import numpy as np
@@ -24,8 +29,8 @@ pytestmark = pytest.mark.gpu
 if torch.cuda.is_available():
     import llama_pre_norm_b200 as lb
 
-# d = 1024 (7 full tiles of the fused QKV rows + 8 of o_proj), f = 2816 (22 tiles of
-# gate/up); weight_std 0.15 makes the branches dominate the residual in y.
+# d = 1024 (12 full tiles of the fused QKV rows, 8 of o_proj), f = 2816 (44 tiles of
+# the interleaved gate/up rows)
 CFG = BlockConfig("w8", d=1024, n_heads=8, n_kv_heads=2, head_dim=128, f=2816, B=4, T=1,
                   dtype="bf16", cache_len=200, weight_std=0.15)
 # ragged everywhere: 5 heads of 64 (QKV rows 960 = 7.5 tiles, d = 320 = 2.5 tiles),
@@ -34,6 +39,18 @@ CFG_RAGGED = BlockConfig("w8-ragged", d=320, n_heads=5, n_kv_heads=5, head_dim=6
                          T=1, dtype="bf16", cache_len=150)
 GROUPS = {"qkv": ("wq", "wk", "wv"), "o": ("wo",), "gate_up": ("w_gate", "w_up"),
           "down": ("w_down",)}
+QK_STD = 0.02
+
+
+def _weights(cfg, seed=0):
+    W = make_weights(cfg, seed=seed)
+    for k in ("wq", "wk"):
+        W[k] = (W[k].double() * (QK_STD / cfg.weight_std)).to(W[k].dtype)
+    return W
+
+
+def _std(cfg, key):
+    return QK_STD if key in ("wq", "wk") else cfg.weight_std
 
 
 def _outliers(w, std):
@@ -96,35 +113,65 @@ def _run(cfg, W, quantize, steps=2, W_after=None):
     return out
 
 
+def _int8_exact(w, gen):
+    """A weight matrix that INT8 represents exactly: w = 2^-9 q, q ~ N(0, 20) rounded
+    and clipped to [-126, 126], one element per row at +-127 (so s = 2^-9 exactly)."""
+    o, i = w.shape
+    q = torch.clamp(torch.round(torch.randn(o, i, generator=gen, dtype=torch.float64) * 20), -126, 126)
+    r = torch.arange(o)
+    q[r, (r * 11) % i] = torch.where(r % 2 == 0, 127.0, -127.0).double()
+    return (q * 2.0 ** -9).to(w.dtype)
+
+
+def test_int8_path_equals_bf16_path_bitwise_on_int8_exact_weights():
+    """On weights with exact INT8 codes and power-of-two row scales the INT8 GEMMs
+    multiply the same products in the same K order as the bf16 GEMMs, and the scale
+    is exact, so the whole decode step must agree bit for bit."""
+    cfg = CFG.with_(weight_std=0.02)
+    W = make_weights(cfg)
+    gen = torch.Generator().manual_seed(77)
+    for k in ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down"):
+        W[k] = _int8_exact(W[k], gen)
+    q8, s8 = ob.quantize_int8_rows(W["w_down"])
+    assert np.all(s8 == np.float32(2.0 ** -9))
+    assert np.array_equal(ob.dequantize_int8_rows(q8, s8), as_np(W["w_down"]))
+    (y16, k16, want), = _run(cfg, W, quantize=False, steps=1)
+    (y8, k8, _), = _run(cfg, W, quantize=True, steps=1)
+    assert torch.equal(k8, k16)
+    assert torch.equal(y8, y16)
+    assert row_err(y8, want["w8"]["y"]) <= BF16_TOL
+
+
 @pytest.mark.parametrize("cfg", [CFG, CFG_RAGGED], ids=lambda c: c.name)
 def test_int8_decode_matches_oracle(cfg):
-    for y, k_new, want in _run(cfg, make_weights(cfg), quantize=True):
+    for y, k_new, want in _run(cfg, _weights(cfg), quantize=True):
         assert row_err(y, want["w8"]["y"]) <= BF16_TOL
         assert row_err(k_new, want["w8"]["k_new"]) <= BF16_TOL
 
 
 @pytest.mark.parametrize("group", list(GROUPS))
 def test_int8_decode_uses_int8_weights_of_each_gemm(group):
-    W = make_weights(CFG)
+    W = _weights(CFG)
     for k in GROUPS[group]:
-        W[k] = _outliers(W[k], CFG.weight_std)
+        W[k] = _outliers(W[k], _std(CFG, k))
     for y, k_new, want in _run(CFG, W, quantize=True, steps=1):
         sep = row_err(want["w8"]["y"], want["bf16"]["y"])
-        assert sep >= 3 * BF16_TOL  # the case separates INT8 from bf16 weights
+        assert sep >= 2 * BF16_TOL  # the case separates INT8 from bf16 weights
         assert row_err(y, want["w8"]["y"]) <= BF16_TOL
-        assert row_err(y, want["bf16"]["y"]) >= 2 * BF16_TOL
+        assert row_err(y, want["bf16"]["y"]) > BF16_TOL
         if group == "qkv":
             assert row_err(k_new, want["w8"]["k_new"]) <= BF16_TOL
 
 
 def test_int8_requantizes_on_set_weights_and_can_be_disabled():
-    W0 = make_weights(CFG)
-    W1 = make_weights(CFG, seed=5)
+    W0 = _weights(CFG)
+    W1 = _weights(CFG, seed=5)
     for k in GROUPS["down"] + GROUPS["qkv"]:
-        W1[k] = _outliers(W1[k], CFG.weight_std)
+        W1[k] = _outliers(W1[k], _std(CFG, k))
     (y, _, want), = _run(CFG, W0, quantize=True, steps=1, W_after=W1)
+    assert row_err(want["w8"]["y"], want["bf16"]["y"]) >= 2 * BF16_TOL
     assert row_err(y, want["w8"]["y"]) <= BF16_TOL
-    assert row_err(y, want["bf16"]["y"]) >= 2 * BF16_TOL
+    assert row_err(y, want["bf16"]["y"]) > BF16_TOL
     # disabled again: the bf16 weights
     (y, _, want), = _run(CFG, W1, quantize=False, steps=1)
     assert row_err(y, want["bf16"]["y"]) <= BF16_TOL
@@ -132,9 +179,10 @@ def test_int8_requantizes_on_set_weights_and_can_be_disabled():
 
 def test_int8_batches_above_32_decode_with_bf16_weights():
     cfg = CFG.with_(B=33, cache_len=64)
-    W = make_weights(cfg)
+    W = _weights(cfg)
     W["w_down"] = _outliers(W["w_down"], cfg.weight_std)
     (y, _, want), = _run(cfg, W, quantize=True, steps=1)
+    assert row_err(want["w8"]["y"], want["bf16"]["y"]) >= 2 * BF16_TOL
     assert row_err(y, want["bf16"]["y"]) <= BF16_TOL
 
 

@@ -10,9 +10,11 @@
 // operand, the B <= 32 tokens the N side, split-K partials) with one more stage:
 //   warp 0      loads: the INT8 weight tile (128 x 64 bytes, one contiguous bulk copy
 //               from the tile-blocked layout) and the bf16 token tile (TMA), a
-//               16-deep ring
-//   warps 6..13 widen the INT8 tile to bf16 (exact: |q| <= 127) straight into TMEM
-//               (tcgen05.st), half a weight row per thread, a 4-deep ring of tiles
+//               12-deep ring whose slots also index the TMEM slots of the widened
+//               tiles, so one tcgen05.commit per K block frees both
+//   warps 6..17 widen the INT8 tile to bf16 (exact: |q| <= 127) straight into TMEM
+//               (tcgen05.st), one weight row per thread; three groups of four warps
+//               take turns over the K blocks
 //   warp 1      tcgen05.mma (M=128, N=32) with the converted tile as the TMEM A operand
 //   warps 2..5  epilogue: partial[split][token][n] = s_n * acc
 #include "common.cuh"
@@ -60,16 +62,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
   return v;
 }
 
-// 16 consecutive 32-bit TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-
 // Four INT8 codes (bytes of u, element j in byte j) to four bf16 (two pairs, element
 // order kept). Each biased byte q + 128 becomes the low byte of the fp32 pattern
 // 0x4B0000xx = 2^23 + q + 128; subtracting 2^23 + 128 leaves q exactly, and since
@@ -86,17 +78,22 @@ __device__ __forceinline__ void i8x4_to_bf16x4(uint32_t u, uint32_t& lo, uint32_
   hi = __byte_perm(__float_as_uint(f2), __float_as_uint(f3), 0x7632);
 }
 
-constexpr int kW8ConvWarps = 8;
+// Converter warps come in groups of four (one per TMEM lane quarter); group g widens
+// the K blocks g, g + G, g + 2G, ... of the CTA's sequence, so G blocks are in flight.
+constexpr int kW8ConvGroups = 3;
+constexpr int kW8ConvWarps = 4 * kW8ConvGroups;
 constexpr int kW8Threads = (6 + kW8ConvWarps) * 32;
 
 template <int BN>
 struct W8Cfg {
-  static constexpr int STAGES = 16;           // load ring: INT8 tile + token tile
-  static constexpr int A_STAGES = 4;          // converted bf16 tiles in TMEM, 32 columns each
+  // One ring index per K block covers its shared-memory slot (INT8 tile + token tile)
+  // and its TMEM slot (the widened tile, 32 columns), so that the MMA issuer frees
+  // both with a single tcgen05.commit per K block.
+  static constexpr int STAGES = 12;
   static constexpr int RAW_BYTES = 128 * 64;  // INT8 weight tile
   static constexpr int B_BYTES = BN * 64 * 2; // bf16 token tile
-  static constexpr int A_COL0 = 2 * BN;       // TMEM: two accumulators, then the A stages
-  static constexpr int TMEM_USED = 2 * BN + A_STAGES * 32;
+  static constexpr int A_COL0 = 2 * BN;       // TMEM: two accumulators, then the A slots
+  static constexpr int TMEM_USED = 2 * BN + STAGES * 32;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
                                    : TMEM_USED <= 256 ? 256 : 512;
   static constexpr int SMEM = STAGES * (RAW_BYTES + B_BYTES) + 512 + 1024;
@@ -108,7 +105,8 @@ __global__ void __launch_bounds__(kW8Threads, 1)
                    const float* __restrict__ row_scale, int M, int N, int K, int kb_per, int n_split,
                    GemmEpi epi) {
   using C = W8Cfg<BN>;
-  constexpr int RS = C::STAGES, AS = C::A_STAGES;
+  constexpr int RS = C::STAGES;
+  static_assert(C::TMEM_USED <= 512, "TMEM");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -116,10 +114,10 @@ __global__ void __launch_bounds__(kW8Threads, 1)
   uint8_t* sRaw = sB + RS * C::B_BYTES;         // RS x 8 KB
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + RS * C::RAW_BYTES);
   uint64_t* full = bars;                // INT8 + token tile landed
-  uint64_t* empty = bars + RS;          // INT8 tile read by the converters, token tile by the MMA
-  uint64_t* a_full = bars + 2 * RS;     // converted tile in TMEM
-  uint64_t* a_empty = a_full + AS;      // converted tile consumed by the MMA
-  uint64_t* tfull = a_empty + AS;
+  uint64_t* raw_free = bars + RS;       // INT8 tile read by its converter group
+  uint64_t* a_full = bars + 2 * RS;     // widened tile in TMEM
+  uint64_t* mma_done = bars + 3 * RS;   // the K block's MMAs completed: token tile and TMEM slot free
+  uint64_t* tfull = bars + 4 * RS;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -128,11 +126,9 @@ __global__ void __launch_bounds__(kW8Threads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < RS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + kW8ConvWarps);  // one MMA commit + every converter warp
-    }
-    for (int s = 0; s < AS; ++s) {
-      mbar_init(&a_full[s], kW8ConvWarps);
-      mbar_init(&a_empty[s], 1);
+      mbar_init(&raw_free[s], 4);  // the four warps of one converter group
+      mbar_init(&a_full[s], 4);
+      mbar_init(&mma_done[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
@@ -164,7 +160,7 @@ __global__ void __launch_bounds__(kW8Threads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- loads
+      // ---------------- loads; slot reuse needs both its INT8 tile read and its MMAs done
       uint32_t stage = 0, phase = 0;
       long long issued = 0;
       bool ok = true;
@@ -172,7 +168,8 @@ __global__ void __launch_bounds__(kW8Threads, 1)
         int mt, nt, sp, kb0, kb1;
         decode(u, mt, nt, sp, kb0, kb1);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, epi.err, 0x41)) {
+          if (!mbar_wait(&raw_free[stage], phase ^ 1, epi.err, 0x41) ||
+              !mbar_wait(&mma_done[stage], phase ^ 1, epi.err, 0x4a)) {
             ok = false;
             break;
           }
@@ -191,13 +188,13 @@ __global__ void __launch_bounds__(kW8Threads, 1)
       pdl_trigger();
       const long long first = issued > RS ? issued - RS : 0;
       for (long long i = first; i < issued; ++i)
-        mbar_wait(&empty[i % RS], (uint32_t)((i / RS) & 1), epi.err, 0x42);
+        mbar_wait(&raw_free[i % RS], (uint32_t)((i / RS) & 1), epi.err, 0x42);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer: A (the converted weights) from TMEM, B from smem
+      // ---------------- MMA issuer: A (the widened weights) from TMEM, B from smem
       constexpr uint32_t idesc = umma_idesc_bf16(128, BN, 0, 0);
-      uint32_t rs = 0, rphase = 0, as = 0, aphase = 0;
+      uint32_t rs = 0, rphase = 0;
       int t = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++t) {
@@ -209,26 +206,21 @@ __global__ void __launch_bounds__(kW8Threads, 1)
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[rs], rphase, epi.err, 0x44) ||
-              !mbar_wait(&a_full[as], aphase, epi.err, 0x45)) {
+              !mbar_wait(&a_full[rs], rphase, epi.err, 0x45)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_tmem = tmem_base + C::A_COL0 + as * 32;
+          const uint32_t a_tmem = tmem_base + C::A_COL0 + rs * 32;
           const uint32_t b0 = smem_u32(sB + rs * C::B_BYTES);
 #pragma unroll
           for (int k = 0; k < 4; ++k)  // K = 16 per MMA: 8 columns of bf16 pairs
             umma_bf16_tmem_a(d_tmem, a_tmem + k * 8, umma_desc_sw128(b0 + k * 32, 16, 1024), idesc,
                              (kb > kb0 || k > 0) ? 1u : 0u);
-          umma_commit(&empty[rs]);
-          umma_commit(&a_empty[as]);
+          umma_commit(&mma_done[rs]);
           if (++rs == RS) {
             rs = 0;
             rphase ^= 1;
-          }
-          if (++as == AS) {
-            as = 0;
-            aphase ^= 1;
           }
         }
         if (!ok) break;
@@ -239,58 +231,64 @@ __global__ void __launch_bounds__(kW8Threads, 1)
     }
   } else if (warp >= 6) {
     // ---------------- INT8 -> bf16 converters. A warp may only reach the TMEM lanes
-    // 32 * (warp % 4) ..+31, so lane l of converter warp w handles weight row
-    // 32 * (w % 4) + l, K half (w - 6) / 4 of the 64-deep block: 32 codes read from
-    // shared memory, widened, stored as 16 columns of bf16 pairs.
-    const int quarter = warp & 3, half = (warp - 6) >> 2;
+    // 32 * (warp % 4) ..+31, so lane l of a group's warp w handles weight row
+    // 32 * (w % 4) + l of the group's K blocks: 64 codes read from shared memory,
+    // widened, stored as 32 columns of bf16 pairs.
+    const int quarter = warp & 3, group = (warp - 6) >> 2;
     const int r = quarter * 32 + lane;
-    // The tile is stored [half][row][32 bytes]; a 16-byte access is served per 8
-    // threads (rows r0..r0+7), on 16-byte bank group 2r + chunk (mod 8): rows with
-    // bit 2 set read their second chunk first, so each phase hits 8 distinct groups.
-    const int first = (r >> 2) & 1;
-    const uint32_t raw0 = smem_u32(sRaw) + half * 4096 + r * 32;
-    const uint32_t lane_addr = ((uint32_t)(quarter * 32) << 16) + C::A_COL0 + half * 16;
-    uint32_t rs = 0, rphase = 0, as = 0, aphase = 0;
+    // The tile is stored [2 K halves][128 rows][32 bytes]; a 16-byte access is served
+    // per 8 threads (rows r0..r0+7), on 16-byte bank group 2r + chunk (mod 8): rows
+    // with bit 2 set read the second chunk of a half first, so each phase hits 8
+    // distinct groups.
+    const int sw = (r >> 2) & 1;
+    const uint32_t raw0 = smem_u32(sRaw) + r * 32;
+    const uint32_t lane_addr = ((uint32_t)(quarter * 32) << 16) + C::A_COL0;
+    long long i = 0;  // position in the CTA's sequence of K blocks
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       int mt, nt, sp, kb0, kb1;
       decode(u, mt, nt, sp, kb0, kb1);
-      for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait_warp(&full[rs], rphase, epi.err, 0x47) ||
-            !mbar_wait_warp(&a_empty[as], aphase ^ 1, epi.err, 0x48)) {
+      for (int kb = kb0; kb < kb1; ++kb, ++i) {
+        if (i % kW8ConvGroups != group) continue;
+        const int rs = (int)(i % RS);
+        const uint32_t ph = (uint32_t)((i / RS) & 1);
+        // the INT8 tile landed, and the slot's previous MMAs no longer read its TMEM
+        if (!mbar_wait_warp(&full[rs], ph, epi.err, 0x47) ||
+            !mbar_wait_warp(&mma_done[rs], ph ^ 1, epi.err, 0x48)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t src = raw0 + rs * C::RAW_BYTES;
-        const uint4 c0 = lds128(src + first * 16);
-        const uint4 c1 = lds128(src + (first ^ 1) * 16);
-        const uint4 lo = first ? c1 : c0, hi = first ? c0 : c1;  // K 0..15, K 16..31 of the half
-        uint32_t p[16];
-        i8x4_to_bf16x4(lo.x, p[0], p[1]);
-        i8x4_to_bf16x4(lo.y, p[2], p[3]);
-        i8x4_to_bf16x4(lo.z, p[4], p[5]);
-        i8x4_to_bf16x4(lo.w, p[6], p[7]);
-        i8x4_to_bf16x4(hi.x, p[8], p[9]);
-        i8x4_to_bf16x4(hi.y, p[10], p[11]);
-        i8x4_to_bf16x4(hi.z, p[12], p[13]);
-        i8x4_to_bf16x4(hi.w, p[14], p[15]);
-        tmem_st16(tmem_base + lane_addr + as * 32, p);
+        const uint4 c00 = lds128(src + sw * 16), c01 = lds128(src + (sw ^ 1) * 16);
+        const uint4 c10 = lds128(src + 4096 + sw * 16), c11 = lds128(src + 4096 + (sw ^ 1) * 16);
+        // K 0..15, 16..31, 32..47, 48..63 of the row
+        const uint4 k0 = sw ? c01 : c00, k1 = sw ? c00 : c01;
+        const uint4 k2 = sw ? c11 : c10, k3 = sw ? c10 : c11;
+        uint32_t p[32];
+        i8x4_to_bf16x4(k0.x, p[0], p[1]);
+        i8x4_to_bf16x4(k0.y, p[2], p[3]);
+        i8x4_to_bf16x4(k0.z, p[4], p[5]);
+        i8x4_to_bf16x4(k0.w, p[6], p[7]);
+        i8x4_to_bf16x4(k1.x, p[8], p[9]);
+        i8x4_to_bf16x4(k1.y, p[10], p[11]);
+        i8x4_to_bf16x4(k1.z, p[12], p[13]);
+        i8x4_to_bf16x4(k1.w, p[14], p[15]);
+        i8x4_to_bf16x4(k2.x, p[16], p[17]);
+        i8x4_to_bf16x4(k2.y, p[18], p[19]);
+        i8x4_to_bf16x4(k2.z, p[20], p[21]);
+        i8x4_to_bf16x4(k2.w, p[22], p[23]);
+        i8x4_to_bf16x4(k3.x, p[24], p[25]);
+        i8x4_to_bf16x4(k3.y, p[26], p[27]);
+        i8x4_to_bf16x4(k3.z, p[28], p[29]);
+        i8x4_to_bf16x4(k3.w, p[30], p[31]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&raw_free[rs]);  // every lane's codes are in registers
+        tmem_st32(tmem_base + lane_addr + rs * 32, reinterpret_cast<const float(&)[32]>(p));
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&a_full[as]);
-          mbar_arrive(&empty[rs]);
-        }
-        if (++rs == RS) {
-          rs = 0;
-          rphase ^= 1;
-        }
-        if (++as == AS) {
-          as = 0;
-          aphase ^= 1;
-        }
+        if (lane == 0) mbar_arrive(&a_full[rs]);
       }
     }
   } else {

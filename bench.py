@@ -40,11 +40,12 @@ UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 CPU_SAMPLE_T = 2048  # tokens of the 7B prefill the CPU oracle evaluates per sample (the full T)
 
-# DRAM traffic per launch of the dominant kernels from ncu captures (see
-# profiles/); None until a capture of the current kernel exists.
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the dominant
+# kernels, from one `ncu --set full` capture of the current kernels on this workload; set
+# to None whenever a kernel changes until it is captured again.
 NCU_TRAFFIC_BYTES = {
-    "gate_up_swiglu_gemm": None,  # kernel changed since profiles/gemm_tc_gate_up_llama7b.md
-    "attention_decode": None,
+    "gate_up_swiglu_gemm": 198_123_776 + 35_764_480,  # gemm_tc_pair_kernel<256, 2>, 7B prefill
+    "attention_decode": 2_148_352_000 + 8_126_464,    # attn_decode_split_kernel<128, 1>, L=4096
 }
 
 

@@ -219,7 +219,9 @@ static int decode_split(int m_tiles, int n_tiles, int bn, int K, int tile_bytes,
 }
 
 // Tile width and split of the four decode GEMMs (QKV, o_proj, gate/up, down) for a
-// batch of B tokens, with the INT8 weights when w8 (used for B <= 32 only).
+// batch of B tokens, with the INT8 weights when w8 (used for B <= 32 only). split[i] is
+// the number of partial slices the GEMM writes (canonical: no two splits give the same
+// units), which the reducing kernel reads.
 struct DecodePlan {
   int bn;
   bool w8;
@@ -231,11 +233,16 @@ static DecodePlan decode_plan(const llama_block* b, int B, bool w8) {
   p.bn = B <= 32 ? 32 : B <= 64 ? 64 : B <= 128 ? 128 : 256;
   p.w8 = w8 && B <= 32;
   const int n_tiles = (B + p.bn - 1) / p.bn;
-  const int tile_bytes = (p.w8 ? 128 * 64 : 128 * 64 * 2) + p.bn * 64 * 2;
   const int M[4] = {b->n_qkv, b->d, b->n_gu, b->d};
   const int K[4] = {b->d, b->H * b->dh, b->d, b->f};
-  for (int i = 0; i < 4; ++i)
-    p.split[i] = decode_split((M[i] + 127) / 128, n_tiles, p.bn, K[i], tile_bytes, b->num_sms);
+  for (int i = 0; i < 4; ++i) {
+    if (p.w8)  // 128-deep K blocks of 16 KB INT8 + the token tile
+      p.split[i] = decode_split((M[i] + 127) / 128, n_tiles, p.bn, (K[i] + 127) / 128 * 64,
+                                128 * 128 + p.bn * 128 * 2, b->num_sms);
+    else
+      p.split[i] = decode_split((M[i] + 127) / 128, n_tiles, p.bn, K[i], 128 * 64 * 2 + p.bn * 64 * 2,
+                                b->num_sms);
+  }
   return p;
 }
 
@@ -675,7 +682,7 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
     const int s1 = plan.split[0];
     LB_STAGE("qkv_gemm", 1, wgemm(0, b->w_qkv, w.h, b->n_qkv, d, s1, e));
     LB_STAGE("qkv_rope_append", 1,
-             launch_qkv_finish(kBF16, w.part, gemm_effective_split(d, s1), e.split_stride, B, 1, H,
+             launch_qkv_finish(kBF16, w.part, s1, e.split_stride, B, 1, H,
                                Hkv, dh, cache_len, 0, b->cos_t, b->sin_t, b->max_pos, w.q, k_cache,
                                v_cache, t_max, b->err, s));
     LB_STAGE("attention", 2, launch_attn_decode(w.q, k_cache, v_cache, w.o, w.attn_part, B, H, Hkv,
@@ -686,19 +693,19 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
     e.ldo = d; e.split_stride = (long long)B * d;
     LB_STAGE("o_proj_gemm", 1, wgemm(1, b->w_o, w.o, d, K2, s2, e));
     LB_STAGE("resid_rmsnorm_mlp", 1,
-             launch_resid_rmsnorm(kBF16, x, w.part, gemm_effective_split(K2, s2), e.split_stride,
+             launch_resid_rmsnorm(kBF16, x, w.part, s2, e.split_stride,
                                   w.x1, nullptr, w.h, B, d, b->eps, s));
     // gate/up (packed rows), SiLU(g) * u
     const int s3 = plan.split[2];
     e.ldo = b->n_gu; e.split_stride = (long long)B * b->n_gu;
     LB_STAGE("gate_up_gemm", 1, wgemm(2, b->w_gu, w.h, b->n_gu, d, s3, e));
-    LB_STAGE("silu_mul", 1, launch_silu_mul(kBF16, w.part, gemm_effective_split(d, s3), e.split_stride,
+    LB_STAGE("silu_mul", 1, launch_silu_mul(kBF16, w.part, s3, e.split_stride,
                                             B, f, b->n_gu, 128, w.a, s));
     // down, y = X' + sum(partials); cache_len += 1
     const int s4 = plan.split[3];
     e.ldo = d; e.split_stride = (long long)B * d;
     LB_STAGE("down_gemm", 1, wgemm(3, b->w_d, w.a, d, f, s4, e));
-    LB_STAGE("resid_add_len", 1, launch_resid_add(kBF16, w.x1, w.part, gemm_effective_split(f, s4),
+    LB_STAGE("resid_add_len", 1, launch_resid_add(kBF16, w.x1, w.part, s4,
                                                   e.split_stride, y, (long long)B * d, cache_len, B,
                                                   1, s));
   } else {

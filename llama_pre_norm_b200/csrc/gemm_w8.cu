@@ -8,10 +8,10 @@
 //
 // The GEMM is the swap-AB decode GEMM of gemm_tc.cu (weights are the 128-row
 // operand, the B <= 32 tokens the N side, split-K partials) with one more stage:
-//   warp 0      loads: the INT8 weight tile (128 x 64 bytes, one contiguous bulk copy
-//               from the tile-blocked layout) and the bf16 token tile (TMA), a
-//               12-deep ring whose slots also index the TMEM slots of the widened
-//               tiles, so one tcgen05.commit per K block frees both
+//   warp 0      loads, per 128-deep K block: the INT8 weight tile (128 x 128 bytes,
+//               one contiguous bulk copy from the tile-blocked layout) and the bf16
+//               token tile (TMA), a 6-deep ring whose slots also index the TMEM slots
+//               of the widened tiles, so one tcgen05.commit per K block frees both
 //   warps 6..17 widen the INT8 tile to bf16 (exact: |q| <= 127) straight into TMEM
 //               (tcgen05.st), one weight row per thread; three groups of four warps
 //               take turns over the K blocks
@@ -86,14 +86,15 @@ constexpr int kW8Threads = (6 + kW8ConvWarps) * 32;
 
 template <int BN>
 struct W8Cfg {
-  // One ring index per K block covers its shared-memory slot (INT8 tile + token tile)
-  // and its TMEM slot (the widened tile, 32 columns), so that the MMA issuer frees
-  // both with a single tcgen05.commit per K block.
-  static constexpr int STAGES = 12;
-  static constexpr int RAW_BYTES = 128 * 64;  // INT8 weight tile
-  static constexpr int B_BYTES = BN * 64 * 2; // bf16 token tile
-  static constexpr int A_COL0 = 2 * BN;       // TMEM: two accumulators, then the A slots
-  static constexpr int TMEM_USED = 2 * BN + STAGES * 32;
+  // One pipeline step covers a 128-deep K block. Its ring index names both its
+  // shared-memory slot (INT8 tile + token tile) and its TMEM slot (the widened tile,
+  // 64 columns), so that the MMA issuer frees both with a single tcgen05.commit.
+  static constexpr int STAGES = 6;
+  static constexpr int RAW_BYTES = 128 * 128;   // INT8 weight tile
+  static constexpr int B_HALF = BN * 64 * 2;    // bf16 token tile, 64 K (one 128-byte swizzle atom)
+  static constexpr int B_BYTES = 2 * B_HALF;
+  static constexpr int A_COL0 = 2 * BN;         // TMEM: two accumulators, then the A slots
+  static constexpr int TMEM_USED = 2 * BN + STAGES * 64;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
                                    : TMEM_USED <= 256 ? 256 : 512;
   static constexpr int SMEM = STAGES * (RAW_BYTES + B_BYTES) + 512 + 1024;
@@ -102,7 +103,7 @@ struct W8Cfg {
 template <int BN>
 __global__ void __launch_bounds__(kW8Threads, 1)
     gemm_w8_kernel(const uint8_t* __restrict__ A8, const __grid_constant__ CUtensorMap tmB,
-                   const float* __restrict__ row_scale, int M, int N, int K, int kb_per, int n_split,
+                   const float* __restrict__ row_scale, int M, int N, int K, int kt_per, int n_split,
                    GemmEpi epi) {
   using C = W8Cfg<BN>;
   constexpr int RS = C::STAGES;
@@ -110,13 +111,13 @@ __global__ void __launch_bounds__(kW8Threads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sB = smem;                           // RS x BN*128 B, 1024-aligned (128-byte swizzle)
-  uint8_t* sRaw = sB + RS * C::B_BYTES;         // RS x 8 KB
+  uint8_t* sB = smem;                           // RS x 2 x BN*128 B, 1024-aligned (128-byte swizzle)
+  uint8_t* sRaw = sB + RS * C::B_BYTES;         // RS x 16 KB
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + RS * C::RAW_BYTES);
   uint64_t* full = bars;                // INT8 + token tile landed
   uint64_t* raw_free = bars + RS;       // INT8 tile read by its converter group
   uint64_t* a_full = bars + 2 * RS;     // widened tile in TMEM
-  uint64_t* mma_done = bars + 3 * RS;   // the K block's MMAs completed: token tile and TMEM slot free
+  uint64_t* mma_done = bars + 3 * RS;   // the block's MMAs completed: token tile and TMEM slot free
   uint64_t* tfull = bars + 4 * RS;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
@@ -146,16 +147,16 @@ __global__ void __launch_bounds__(kW8Threads, 1)
   pdl_wait();
 
   const int num_m = (M + 127) / 128, num_n = (N + BN - 1) / BN;
-  const int KB = (K + 63) / 64;
+  const int KT = (K + 127) / 128;
   const int units = num_m * num_n * n_split;
-  auto decode = [&](int u, int& mt, int& nt, int& sp, int& kb0, int& kb1) {
+  auto decode = [&](int u, int& mt, int& nt, int& sp, int& kt0, int& kt1) {
     const int mn = num_m * num_n;
     sp = u / mn;
     const int rem = u - sp * mn;
     mt = rem % num_m;
     nt = rem / num_m;
-    kb0 = sp * kb_per;
-    kb1 = min(KB, kb0 + kb_per);
+    kt0 = sp * kt_per;
+    kt1 = min(KT, kt0 + kt_per);
   };
 
   if (warp == 0) {
@@ -165,19 +166,22 @@ __global__ void __launch_bounds__(kW8Threads, 1)
       long long issued = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        int mt, nt, sp, kb0, kb1;
-        decode(u, mt, nt, sp, kb0, kb1);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        int mt, nt, sp, kt0, kt1;
+        decode(u, mt, nt, sp, kt0, kt1);
+        for (int kt = kt0; kt < kt1; ++kt) {
           if (!mbar_wait(&raw_free[stage], phase ^ 1, epi.err, 0x41) ||
               !mbar_wait(&mma_done[stage], phase ^ 1, epi.err, 0x4a)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&full[stage], C::RAW_BYTES + C::B_BYTES);
-          // one contiguous 8 KB tile of the blocked layout
-          bulk_load(sRaw + stage * C::RAW_BYTES, A8 + ((long long)mt * KB + kb) * C::RAW_BYTES,
+          // one contiguous 16 KB tile of the blocked layout
+          bulk_load(sRaw + stage * C::RAW_BYTES, A8 + ((long long)mt * KT + kt) * C::RAW_BYTES,
                     C::RAW_BYTES, &full[stage]);
-          tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * 64, nt * BN);
+          // the token tile as two 64-deep halves (past K they read as zeros)
+          uint8_t* b = sB + stage * C::B_BYTES;
+          tma_load_2d(b, &tmB, &full[stage], kt * 128, nt * BN);
+          tma_load_2d(b + C::B_HALF, &tmB, &full[stage], kt * 128 + 64, nt * BN);
           ++issued;
           if (++stage == RS) {
             stage = 0;
@@ -198,25 +202,26 @@ __global__ void __launch_bounds__(kW8Threads, 1)
       int t = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++t) {
-        int mt, nt, sp, kb0, kb1;
-        decode(u, mt, nt, sp, kb0, kb1);
+        int mt, nt, sp, kt0, kt1;
+        decode(u, mt, nt, sp, kt0, kt1);
         const int acc = t & 1;
         if (!mbar_wait(&tempty[acc], ((t >> 1) & 1) ^ 1, epi.err, 0x43)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kt = kt0; kt < kt1; ++kt) {
           if (!mbar_wait(&full[rs], rphase, epi.err, 0x44) ||
               !mbar_wait(&a_full[rs], rphase, epi.err, 0x45)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_tmem = tmem_base + C::A_COL0 + rs * 32;
+          const uint32_t a_tmem = tmem_base + C::A_COL0 + rs * 64;
           const uint32_t b0 = smem_u32(sB + rs * C::B_BYTES);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)  // K = 16 per MMA: 8 columns of bf16 pairs
-            umma_bf16_tmem_a(d_tmem, a_tmem + k * 8, umma_desc_sw128(b0 + k * 32, 16, 1024), idesc,
-                             (kb > kb0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 8; ++k)  // K = 16 per MMA: 8 TMEM columns of bf16 pairs
+            umma_bf16_tmem_a(d_tmem, a_tmem + k * 8,
+                             umma_desc_sw128(b0 + (k >> 2) * C::B_HALF + (k & 3) * 32, 16, 1024), idesc,
+                             (kt > kt0 || k > 0) ? 1u : 0u);
           umma_commit(&mma_done[rs]);
           if (++rs == RS) {
             rs = 0;
@@ -232,23 +237,23 @@ __global__ void __launch_bounds__(kW8Threads, 1)
   } else if (warp >= 6) {
     // ---------------- INT8 -> bf16 converters. A warp may only reach the TMEM lanes
     // 32 * (warp % 4) ..+31, so lane l of a group's warp w handles weight row
-    // 32 * (w % 4) + l of the group's K blocks: 64 codes read from shared memory,
-    // widened, stored as 32 columns of bf16 pairs.
+    // 32 * (w % 4) + l of the group's K blocks: 128 codes read from shared memory,
+    // widened, stored as 64 columns of bf16 pairs.
     const int quarter = warp & 3, group = (warp - 6) >> 2;
     const int r = quarter * 32 + lane;
-    // The tile is stored [2 K halves][128 rows][32 bytes]; a 16-byte access is served
-    // per 8 threads (rows r0..r0+7), on 16-byte bank group 2r + chunk (mod 8): rows
-    // with bit 2 set read the second chunk of a half first, so each phase hits 8
-    // distinct groups.
+    // The tile is stored [4 K quarters][128 rows][32 bytes]; a 16-byte access is served
+    // per 8 threads (rows r0..r0+7), on 16-byte bank group 2r + chunk (mod 8): rows with
+    // bit 2 set read the second chunk of a quarter first, so each phase hits 8 distinct
+    // groups.
     const int sw = (r >> 2) & 1;
     const uint32_t raw0 = smem_u32(sRaw) + r * 32;
     const uint32_t lane_addr = ((uint32_t)(quarter * 32) << 16) + C::A_COL0;
     long long i = 0;  // position in the CTA's sequence of K blocks
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-      int mt, nt, sp, kb0, kb1;
-      decode(u, mt, nt, sp, kb0, kb1);
-      for (int kb = kb0; kb < kb1; ++kb, ++i) {
+      int mt, nt, sp, kt0, kt1;
+      decode(u, mt, nt, sp, kt0, kt1);
+      for (int kt = kt0; kt < kt1; ++kt, ++i) {
         if (i % kW8ConvGroups != group) continue;
         const int rs = (int)(i % RS);
         const uint32_t ph = (uint32_t)((i / RS) & 1);
@@ -260,31 +265,35 @@ __global__ void __launch_bounds__(kW8Threads, 1)
         }
         tc_fence_after();
         const uint32_t src = raw0 + rs * C::RAW_BYTES;
-        const uint4 c00 = lds128(src + sw * 16), c01 = lds128(src + (sw ^ 1) * 16);
-        const uint4 c10 = lds128(src + 4096 + sw * 16), c11 = lds128(src + 4096 + (sw ^ 1) * 16);
-        // K 0..15, 16..31, 32..47, 48..63 of the row
-        const uint4 k0 = sw ? c01 : c00, k1 = sw ? c00 : c01;
-        const uint4 k2 = sw ? c11 : c10, k3 = sw ? c10 : c11;
-        uint32_t p[32];
-        i8x4_to_bf16x4(k0.x, p[0], p[1]);
-        i8x4_to_bf16x4(k0.y, p[2], p[3]);
-        i8x4_to_bf16x4(k0.z, p[4], p[5]);
-        i8x4_to_bf16x4(k0.w, p[6], p[7]);
-        i8x4_to_bf16x4(k1.x, p[8], p[9]);
-        i8x4_to_bf16x4(k1.y, p[10], p[11]);
-        i8x4_to_bf16x4(k1.z, p[12], p[13]);
-        i8x4_to_bf16x4(k1.w, p[14], p[15]);
-        i8x4_to_bf16x4(k2.x, p[16], p[17]);
-        i8x4_to_bf16x4(k2.y, p[18], p[19]);
-        i8x4_to_bf16x4(k2.z, p[20], p[21]);
-        i8x4_to_bf16x4(k2.w, p[22], p[23]);
-        i8x4_to_bf16x4(k3.x, p[24], p[25]);
-        i8x4_to_bf16x4(k3.y, p[26], p[27]);
-        i8x4_to_bf16x4(k3.z, p[28], p[29]);
-        i8x4_to_bf16x4(k3.w, p[30], p[31]);
+        const uint32_t dst = tmem_base + lane_addr + rs * 64;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {  // K 0..63, then K 64..127
+          const uint32_t q0 = src + (2 * hh) * 4096, q1 = q0 + 4096;
+          const uint4 c00 = lds128(q0 + sw * 16), c01 = lds128(q0 + (sw ^ 1) * 16);
+          const uint4 c10 = lds128(q1 + sw * 16), c11 = lds128(q1 + (sw ^ 1) * 16);
+          const uint4 k0 = sw ? c01 : c00, k1 = sw ? c00 : c01;
+          const uint4 k2 = sw ? c11 : c10, k3 = sw ? c10 : c11;
+          uint32_t p[32];
+          i8x4_to_bf16x4(k0.x, p[0], p[1]);
+          i8x4_to_bf16x4(k0.y, p[2], p[3]);
+          i8x4_to_bf16x4(k0.z, p[4], p[5]);
+          i8x4_to_bf16x4(k0.w, p[6], p[7]);
+          i8x4_to_bf16x4(k1.x, p[8], p[9]);
+          i8x4_to_bf16x4(k1.y, p[10], p[11]);
+          i8x4_to_bf16x4(k1.z, p[12], p[13]);
+          i8x4_to_bf16x4(k1.w, p[14], p[15]);
+          i8x4_to_bf16x4(k2.x, p[16], p[17]);
+          i8x4_to_bf16x4(k2.y, p[18], p[19]);
+          i8x4_to_bf16x4(k2.z, p[20], p[21]);
+          i8x4_to_bf16x4(k2.w, p[22], p[23]);
+          i8x4_to_bf16x4(k3.x, p[24], p[25]);
+          i8x4_to_bf16x4(k3.y, p[26], p[27]);
+          i8x4_to_bf16x4(k3.z, p[28], p[29]);
+          i8x4_to_bf16x4(k3.w, p[30], p[31]);
+          tmem_st32(dst + hh * 32, reinterpret_cast<const float(&)[32]>(p));
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&raw_free[rs]);  // every lane's codes are in registers
-        tmem_st32(tmem_base + lane_addr + rs * 32, reinterpret_cast<const float(&)[32]>(p));
+        if (lane == 0) mbar_arrive(&raw_free[rs]);  // every lane's codes are consumed
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -297,8 +306,8 @@ __global__ void __launch_bounds__(kW8Threads, 1)
     const int row_in_tile = quarter * 32 + lane;
     int t = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++t) {
-      int mt, nt, sp, kb0, kb1;
-      decode(u, mt, nt, sp, kb0, kb1);
+      int mt, nt, sp, kt0, kt1;
+      decode(u, mt, nt, sp, kt0, kt1);
       const int acc = t & 1;
       if (!mbar_wait_warp(&tfull[acc], (t >> 1) & 1, epi.err, 0x49)) break;
       tc_fence_after();
@@ -342,9 +351,9 @@ cudaError_t launch_gemm_w8(const void* A8, const float* row_scale, const void* B
   CUtensorMap tb;
   if (reinterpret_cast<uintptr_t>(A8) & 15) return cudaErrorInvalidValue;
   if (!make_tmap_2d_bf16(&tb, B, (uint64_t)N, (uint64_t)K, BN)) return cudaErrorInvalidValue;
-  const int KB = K / 64;
-  n_split = gemm_effective_split(K, n_split);
-  const int kb_per = (KB + n_split - 1) / n_split;
+  const int KT = (K + 127) / 128;
+  n_split = w8_effective_split(K, n_split);
+  const int kt_per = (KT + n_split - 1) / n_split;
   const long long units = (long long)((M + 127) / 128) * n_split;
   const int grid = (int)std::min<long long>(units, num_sms);
   auto kern = gemm_w8_kernel<BN>;
@@ -355,7 +364,7 @@ cudaError_t launch_gemm_w8(const void* A8, const float* row_scale, const void* B
     attr_set = true;
   }
   return launch_k(kern, grid, kW8Threads, C::SMEM, s, (const uint8_t*)A8, tb, row_scale, M, N, K,
-                  kb_per, n_split, epi);
+                  kt_per, n_split, epi);
 }
 
 }  // namespace lb

@@ -145,21 +145,30 @@ cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, in
                            const GemmEpi& epi, int num_sms, cudaStream_t s);
 
 // ----------------------------------------------------------- gemm_w8.cu (INT8 weights, decode)
-// INT8 codes are stored tile-blocked so that a decode GEMM streams each 128 x 64 tile
-// as one contiguous 8 KB run, [ceil(rows/128)][cols/64] tiles (cols % 64 == 0, rows
-// padded to a multiple of 128 with zero codes), each tile [2 halves of K][128 rows][32].
+// INT8 codes are stored tile-blocked so that a decode GEMM streams each 128 x 128 tile
+// as one contiguous 16 KB run: [ceil(rows/128)][ceil(cols/128)] tiles (rows and cols
+// padded to multiples of 128 with zero codes), each tile [4 K quarters][128 rows][32].
 __host__ __device__ inline long long w8_blocked_offset(int row, int col, int cols) {
-  return ((long long)(row >> 7) * (cols >> 6) + (col >> 6)) * 8192 + ((col >> 5) & 1) * 4096 +
-         (row & 127) * 32 + (col & 31);
+  const long long tile = (long long)(row >> 7) * ((cols + 127) >> 7) + (col >> 7);
+  return tile * 16384 + ((col >> 5) & 3) * 4096 + (row & 127) * 32 + (col & 31);
 }
-inline size_t w8_blocked_bytes(int rows, int cols) { return (size_t)((rows + 127) / 128) * 128 * cols; }
+inline size_t w8_blocked_bytes(int rows, int cols) {
+  return (size_t)((rows + 127) / 128) * 128 * (size_t)((cols + 127) / 128) * 128;
+}
+// Split-K slices of an INT8 decode GEMM over K (in 128-deep blocks) for a requested split.
+inline int w8_effective_split(int K, int n_split) {
+  const int KT = (K + 127) / 128;
+  n_split = std::max(1, std::min(n_split, KT));
+  const int per = (KT + n_split - 1) / n_split;
+  return (KT + per - 1) / per;
+}
 // q = rint(w / s_r), s_r = max_c |w[r][c]| / 127 (fp32), bf16 w [rows, cols] -> blocked q
 // (zeroed beforehand by the caller), scale[rows].
 cudaError_t launch_quantize_rows_int8(const void* w, void* q, float* scale, int rows, int cols,
                                       cudaStream_t s);
 // Swap-AB decode GEMM with blocked INT8 weights A8 (M rows, row scales row_scale[M]) and
 // bf16 tokens B [N <= 32, K]: part[split][token][row] = row_scale[row] * sum_k A8 B
-// (kEpiPartialT layout). K % 64 == 0.
+// (kEpiPartialT layout), w8_effective_split(K, n_split) slices. K % 64 == 0.
 cudaError_t launch_gemm_w8(const void* A8, const float* row_scale, const void* B, int M, int N,
                            int K, int n_split, const GemmEpi& epi, int num_sms, cudaStream_t s);
 

@@ -8,8 +8,8 @@ the bf16 tolerance, so agreement with the INT8 oracle does not show that the INT
 weights were used. The per-GEMM cases therefore plant one outlier per row in one
 weight group (each row's outlier in a different column), which makes the INT8 and
 the bf16 results of the oracle differ by two tolerances or more; the GPU must match
-the INT8 one and miss the bf16 one. A further case makes both paths compute the same
-products exactly and asks for bit equality.
+the INT8 one and miss the bf16 one. A further case makes both paths form the same
+products exactly and asks for agreement to the rounding of the outputs.
 
 The projections have std 0.15 so that the branches, not the residual, dominate y;
 W_q and W_k keep std 0.02, since larger q and k make the softmax so sharp that bf16
@@ -123,10 +123,11 @@ def _int8_exact(w, gen):
     return (q * 2.0 ** -9).to(w.dtype)
 
 
-def test_int8_path_equals_bf16_path_bitwise_on_int8_exact_weights():
-    """On weights with exact INT8 codes and power-of-two row scales the INT8 GEMMs
-    multiply the same products in the same K order as the bf16 GEMMs, and the scale
-    is exact, so the whole decode step must agree bit for bit."""
+def test_int8_path_matches_bf16_path_on_int8_exact_weights():
+    """On weights with exact INT8 codes and power-of-two row scales the INT8 GEMMs form
+    the same products as the bf16 GEMMs and the scale is exact; only the fp32 summation
+    order may differ (the INT8 GEMM splits K in 128-deep blocks, the bf16 one in 64-deep
+    blocks). So every stored K row agrees to one bf16 rounding, and y to a few."""
     cfg = CFG.with_(weight_std=0.02)
     W = make_weights(cfg)
     gen = torch.Generator().manual_seed(77)
@@ -137,8 +138,10 @@ def test_int8_path_equals_bf16_path_bitwise_on_int8_exact_weights():
     assert np.array_equal(ob.dequantize_int8_rows(q8, s8), as_np(W["w_down"]))
     (y16, k16, want), = _run(cfg, W, quantize=False, steps=1)
     (y8, k8, _), = _run(cfg, W, quantize=True, steps=1)
-    assert torch.equal(k8, k16)
-    assert torch.equal(y8, y16)
+    ulp = 2.0 ** -7  # relative spacing bound of bf16 normals
+    assert torch.all((k8.float() - k16.float()).abs() <= ulp * k16.float().abs() + 1e-30)
+    assert row_err(y8, y16.double().cpu().numpy()) <= 4e-3
+    assert (y8 == y16).double().mean().item() >= 0.5
     assert row_err(y8, want["w8"]["y"]) <= BF16_TOL
 
 

@@ -236,9 +236,9 @@ static DecodePlan decode_plan(const llama_block* b, int B, bool w8) {
   const int M[4] = {b->n_qkv, b->d, b->n_gu, b->d};
   const int K[4] = {b->d, b->H * b->dh, b->d, b->f};
   for (int i = 0; i < 4; ++i) {
-    if (p.w8)  // 128-deep K blocks of 16 KB INT8 + the token tile
-      p.split[i] = decode_split((M[i] + 127) / 128, n_tiles, p.bn, (K[i] + 127) / 128 * 64,
-                                128 * 128 + p.bn * 128 * 2, b->num_sms);
+    if (p.w8)  // kW8K-deep K blocks of INT8 + the token tile
+      p.split[i] = decode_split((M[i] + 127) / 128, n_tiles, p.bn, (K[i] + kW8K - 1) / kW8K * 64,
+                                128 * kW8K + p.bn * kW8K * 2, b->num_sms);
     else
       p.split[i] = decode_split((M[i] + 127) / 128, n_tiles, p.bn, K[i], 128 * 64 * 2 + p.bn * 64 * 2,
                                 b->num_sms);

@@ -8,9 +8,9 @@
 //
 // The GEMM is the swap-AB decode GEMM of gemm_tc.cu (weights are the 128-row
 // operand, the B <= 32 tokens the N side, split-K partials) with one more stage:
-//   warp 0      loads, per 128-deep K block: the INT8 weight tile (128 x 128 bytes,
-//               one contiguous bulk copy from the tile-blocked layout) and the bf16
-//               token tile (TMA), a 6-deep ring whose slots also index the TMEM slots
+//   warp 0      loads, per kW8K-deep K block (kW8K = 128): the INT8 weight tile (128 x
+//               kW8K bytes, one contiguous bulk copy from the tile-blocked layout) and
+//               the bf16 token tile (TMA), a ring whose slots also index the TMEM slots
 //               of the widened tiles, so one tcgen05.commit per K block frees both
 //   warps 6..17 widen the INT8 tile to bf16 (exact: |q| <= 127) straight into TMEM
 //               (tcgen05.st), one weight row per thread; three groups of four warps
@@ -86,15 +86,17 @@ constexpr int kW8Threads = (6 + kW8ConvWarps) * 32;
 
 template <int BN>
 struct W8Cfg {
-  // One pipeline step covers a 128-deep K block. Its ring index names both its
+  // One pipeline step covers a kW8K-deep K block. Its ring index names both its
   // shared-memory slot (INT8 tile + token tile) and its TMEM slot (the widened tile,
-  // 64 columns), so that the MMA issuer frees both with a single tcgen05.commit.
-  static constexpr int STAGES = 6;
-  static constexpr int RAW_BYTES = 128 * 128;   // INT8 weight tile
-  static constexpr int B_HALF = BN * 64 * 2;    // bf16 token tile, 64 K (one 128-byte swizzle atom)
-  static constexpr int B_BYTES = 2 * B_HALF;
-  static constexpr int A_COL0 = 2 * BN;         // TMEM: two accumulators, then the A slots
-  static constexpr int TMEM_USED = 2 * BN + STAGES * 64;
+  // kW8K/2 columns), so that the MMA issuer frees both with a single tcgen05.commit.
+  static constexpr int HALVES = kW8K / 64;       // 64-deep pieces of a step
+  static constexpr int A_COLS = kW8K / 2;        // TMEM columns of one widened tile
+  static constexpr int STAGES = (512 - 2 * BN) / A_COLS < 6 ? (512 - 2 * BN) / A_COLS : 6;
+  static constexpr int RAW_BYTES = 128 * kW8K;   // INT8 weight tile
+  static constexpr int B_HALF = BN * 64 * 2;     // bf16 token tile, 64 K (one 128-byte swizzle atom)
+  static constexpr int B_BYTES = HALVES * B_HALF;
+  static constexpr int A_COL0 = 2 * BN;          // TMEM: two accumulators, then the A slots
+  static constexpr int TMEM_USED = 2 * BN + STAGES * A_COLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
                                    : TMEM_USED <= 256 ? 256 : 512;
   static constexpr int SMEM = STAGES * (RAW_BYTES + B_BYTES) + 512 + 1024;
@@ -147,7 +149,7 @@ __global__ void __launch_bounds__(kW8Threads, 1)
   pdl_wait();
 
   const int num_m = (M + 127) / 128, num_n = (N + BN - 1) / BN;
-  const int KT = (K + 127) / 128;
+  const int KT = (K + kW8K - 1) / kW8K;
   const int units = num_m * num_n * n_split;
   auto decode = [&](int u, int& mt, int& nt, int& sp, int& kt0, int& kt1) {
     const int mn = num_m * num_n;
@@ -175,13 +177,14 @@ __global__ void __launch_bounds__(kW8Threads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[stage], C::RAW_BYTES + C::B_BYTES);
-          // one contiguous 16 KB tile of the blocked layout
+          // one contiguous tile of the blocked layout
           bulk_load(sRaw + stage * C::RAW_BYTES, A8 + ((long long)mt * KT + kt) * C::RAW_BYTES,
                     C::RAW_BYTES, &full[stage]);
-          // the token tile as two 64-deep halves (past K they read as zeros)
+          // the token tile in 64-deep pieces (past K they read as zeros)
           uint8_t* b = sB + stage * C::B_BYTES;
-          tma_load_2d(b, &tmB, &full[stage], kt * 128, nt * BN);
-          tma_load_2d(b + C::B_HALF, &tmB, &full[stage], kt * 128 + 64, nt * BN);
+#pragma unroll
+          for (int hh = 0; hh < C::HALVES; ++hh)
+            tma_load_2d(b + hh * C::B_HALF, &tmB, &full[stage], kt * kW8K + hh * 64, nt * BN);
           ++issued;
           if (++stage == RS) {
             stage = 0;
@@ -215,10 +218,10 @@ __global__ void __launch_bounds__(kW8Threads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_tmem = tmem_base + C::A_COL0 + rs * 64;
+          const uint32_t a_tmem = tmem_base + C::A_COL0 + rs * C::A_COLS;
           const uint32_t b0 = smem_u32(sB + rs * C::B_BYTES);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)  // K = 16 per MMA: 8 TMEM columns of bf16 pairs
+          for (int k = 0; k < kW8K / 16; ++k)  // K = 16 per MMA: 8 TMEM columns of bf16 pairs
             umma_bf16_tmem_a(d_tmem, a_tmem + k * 8,
                              umma_desc_sw128(b0 + (k >> 2) * C::B_HALF + (k & 3) * 32, 16, 1024), idesc,
                              (kt > kt0 || k > 0) ? 1u : 0u);
@@ -237,8 +240,8 @@ __global__ void __launch_bounds__(kW8Threads, 1)
   } else if (warp >= 6) {
     // ---------------- INT8 -> bf16 converters. A warp may only reach the TMEM lanes
     // 32 * (warp % 4) ..+31, so lane l of a group's warp w handles weight row
-    // 32 * (w % 4) + l of the group's K blocks: 128 codes read from shared memory,
-    // widened, stored as 64 columns of bf16 pairs.
+    // 32 * (w % 4) + l of the group's K blocks: kW8K codes read from shared memory,
+    // widened, stored as kW8K/2 columns of bf16 pairs.
     const int quarter = warp & 3, group = (warp - 6) >> 2;
     const int r = quarter * 32 + lane;
     // The tile is stored [4 K quarters][128 rows][32 bytes]; a 16-byte access is served
@@ -265,9 +268,9 @@ __global__ void __launch_bounds__(kW8Threads, 1)
         }
         tc_fence_after();
         const uint32_t src = raw0 + rs * C::RAW_BYTES;
-        const uint32_t dst = tmem_base + lane_addr + rs * 64;
+        const uint32_t dst = tmem_base + lane_addr + rs * C::A_COLS;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {  // K 0..63, then K 64..127
+        for (int hh = 0; hh < C::HALVES; ++hh) {  // K 64*hh .. 64*hh+63
           const uint32_t q0 = src + (2 * hh) * 4096, q1 = q0 + 4096;
           const uint4 c00 = lds128(q0 + sw * 16), c01 = lds128(q0 + (sw ^ 1) * 16);
           const uint4 c10 = lds128(q1 + sw * 16), c11 = lds128(q1 + (sw ^ 1) * 16);
@@ -351,7 +354,7 @@ cudaError_t launch_gemm_w8(const void* A8, const float* row_scale, const void* B
   CUtensorMap tb;
   if (reinterpret_cast<uintptr_t>(A8) & 15) return cudaErrorInvalidValue;
   if (!make_tmap_2d_bf16(&tb, B, (uint64_t)N, (uint64_t)K, BN)) return cudaErrorInvalidValue;
-  const int KT = (K + 127) / 128;
+  const int KT = (K + kW8K - 1) / kW8K;
   n_split = w8_effective_split(K, n_split);
   const int kt_per = (KT + n_split - 1) / n_split;
   const long long units = (long long)((M + 127) / 128) * n_split;

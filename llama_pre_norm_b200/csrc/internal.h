@@ -145,19 +145,22 @@ cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, in
                            const GemmEpi& epi, int num_sms, cudaStream_t s);
 
 // ----------------------------------------------------------- gemm_w8.cu (INT8 weights, decode)
-// INT8 codes are stored tile-blocked so that a decode GEMM streams each 128 x 128 tile
-// as one contiguous 16 KB run: [ceil(rows/128)][ceil(cols/128)] tiles (rows and cols
-// padded to multiples of 128 with zero codes), each tile [4 K quarters][128 rows][32].
+// Depth (K elements) of one pipeline step of the INT8 decode GEMM, and of one tile of
+// the blocked INT8 layout.
+constexpr int kW8K = 128;
+// INT8 codes are stored tile-blocked so that a decode GEMM streams each 128 x kW8K tile
+// as one contiguous run: [ceil(rows/128)][ceil(cols/kW8K)] tiles (rows and cols padded
+// with zero codes), each tile [kW8K/32 K quarters][128 rows][32].
 __host__ __device__ inline long long w8_blocked_offset(int row, int col, int cols) {
-  const long long tile = (long long)(row >> 7) * ((cols + 127) >> 7) + (col >> 7);
-  return tile * 16384 + ((col >> 5) & 3) * 4096 + (row & 127) * 32 + (col & 31);
+  const long long tile = (long long)(row >> 7) * ((cols + kW8K - 1) / kW8K) + col / kW8K;
+  return tile * (128 * kW8K) + ((col % kW8K) >> 5) * 4096 + (row & 127) * 32 + (col & 31);
 }
 inline size_t w8_blocked_bytes(int rows, int cols) {
-  return (size_t)((rows + 127) / 128) * 128 * (size_t)((cols + 127) / 128) * 128;
+  return (size_t)((rows + 127) / 128) * 128 * (size_t)((cols + kW8K - 1) / kW8K) * kW8K;
 }
-// Split-K slices of an INT8 decode GEMM over K (in 128-deep blocks) for a requested split.
+// Split-K slices of an INT8 decode GEMM over K (in kW8K-deep blocks) for a requested split.
 inline int w8_effective_split(int K, int n_split) {
-  const int KT = (K + 127) / 128;
+  const int KT = (K + kW8K - 1) / kW8K;
   n_split = std::max(1, std::min(n_split, KT));
   const int per = (KT + n_split - 1) / n_split;
   return (KT + per - 1) / per;

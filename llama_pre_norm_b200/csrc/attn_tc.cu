@@ -19,8 +19,10 @@
 //                S_t(j+1) overwrites P_t(j), so it is issued only after PV_t(j) has
 //                completed; with two tiles in flight that wait leaves no bubble.
 //   warps 2..5   softmax of tile A, warps 6..9 softmax of tile B: one query row per
-//                thread (= TMEM lane); online max/sum in fp32 with ex2 and
-//                log2(e)/sqrt(d_h) folded into the scale. The running max is only
+//                thread (= TMEM lane); online max/sum in fp32 with log2(e)/sqrt(d_h)
+//                folded into the exponent's FMA and a three-input max (measured:
+//                packed f32x2 forms and an FMA-pipe polynomial for part of the
+//                exponentials were slower here). The running max is only
 //                moved (and O rescaled in TMEM) when a row's max grows by more than
 //                2^8, so most tiles skip the rescale; P <= 2^8 stays exact enough in
 //                bf16 and the final O / l uses the same reference max.
@@ -33,6 +35,14 @@ namespace lb {
 
 constexpr int kAttnTcThreads = 320;
 constexpr float kRescaleLog2 = 8.0f;
+
+// ---------------------------------------------------------------- softmax arithmetic
+// Three-input max (sm_100): one instruction per two new scores.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 template <int DH>
 struct AttnCfg {
@@ -217,49 +227,51 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
         break;
       }
       tc_fence_after();
+      const bool need_mask = j * C::BKV + C::BKV - 1 > off + row0;  // uniform in the CTA
       float s[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, s[c]);
       tmem_wait_ld();
-      const bool need_mask = j * C::BKV + C::BKV - 1 > off + row0;
-      float mx = -INFINITY;
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (j * C::BKV + c * 32 + i > qp) s[c][i] = -INFINITY;
+      }
+      // row max of the raw scores (the scale is positive), three at a time
+      float mxr = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float v = s[c][i] * scale_log2;
-          if (need_mask && j * C::BKV + c * 32 + i > qp) v = -INFINITY;
-          s[c][i] = v;
-          mx = fmaxf(mx, v);
-        }
+        for (int i = 0; i < 32; i += 2) mxr = max3(mxr, s[c][i], s[c][i + 1]);
+      const float mx = mxr * scale_log2;
       // Move the reference max only when this row's max grew by more than 2^8
       // (always on the first tile, where the reference is still -inf).
       const bool move = mx > m_ref + kRescaleLog2;
       const float m_new = move ? mx : m_ref;
       const float alpha = move ? ex2_approx(m_ref - m_new) : 1.f;  // 0 on the first tile
-      float rs = 0.f;
+      // p = 2^(s * scale - m): the scale folded into one FMA per key, the row sum in two
+      // independent accumulators. P is packed in place as bf16 pairs (word k of chunk c:
+      // keys 32c + 2k, 32c + 2k + 1, over elements already consumed) and stored over
+      // the first 64 score columns (column c: keys 2c, 2c+1); keys 32c.. land in
+      // columns 16c.., whose scores are already in registers.
+      const float nm = -m_new;
+      float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 4; ++c) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p = ex2_approx(s[c][i] - m_new);
-          s[c][i] = p;
-          rs += p;
+        for (int i = 0; i < 32; i += 2) {
+          const float p0 = ex2_approx(fmaf(s[c][i], scale_log2, nm));
+          const float p1 = ex2_approx(fmaf(s[c][i + 1], scale_log2, nm));
+          rs0 += p0;
+          rs1 += p1;
+          s[c][i >> 1] = __uint_as_float(pack_bf16x2(p0, p1));
         }
-      l_run = l_run * alpha + rs;
-      m_ref = m_new;
-      // P_t as bf16 pairs over the first 64 score columns (column c: keys 2c, 2c+1),
-      // packed in place: keys 0..63 into s[0], keys 64..127 into s[2].
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float* lo = s[2 * hh];
-        float* hi = s[2 * hh + 1];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) lo[i] = __uint_as_float(pack_bf16x2(lo[2 * i], lo[2 * i + 1]));
-#pragma unroll
-        for (int i = 0; i < 16; ++i) lo[16 + i] = __uint_as_float(pack_bf16x2(hi[2 * i], hi[2 * i + 1]));
-        tmem_st32(t_s + hh * 32, s[2 * hh]);
+        tmem_st16(t_s + c * 16, *reinterpret_cast<const uint32_t(*)[16]>(s[c]));
       }
+      l_run = l_run * alpha + (rs0 + rs1);
+      m_ref = m_new;
       if (j > 0 && __any_sync(0xffffffffu, move)) {
         // O_t holds PV_t(j-1) in full (S_t(j) was issued after it completed); it is
         // rescaled before this tile's P is released to the MMA.

@@ -3,8 +3,8 @@ times (the handle's prefill / decode through the C ABI, bf16):
 
   * LLaMA-7B-shaped prefill (B=1, T=2048), 13B-shaped (B=4, T=1024) and the
     70B-shaped GQA block (64 query / 8 KV heads, T=4096),
-  * one KV-cache decode step of the 7B-shaped block with B=32 and 4096 cached
-    positions.
+  * two KV-cache decode steps of the 7B-, 13B- and 70B-shaped blocks with B=32 and
+    4096 cached positions, and of the 7B-shaped block with INT8 weights.
 
 The oracle evaluates sampled outputs: 64 token rows per sequence (first, last
 and 62 seeded-random rows; K and V are projected for every token since
@@ -52,21 +52,37 @@ def test_full_size_prefill_sampled_rows(cfg):
     blk.close()
 
 
-def test_full_size_decode_step():
-    cfg = DECODE7B
-    t_max = cfg.cache_len + cfg.decode_steps
+DECODE_CFGS = [
+    DECODE7B,
+    # the 13B and the 70B GQA blocks in the same decode setting (B=32, 4096 cached
+    # positions); the 70B one runs the n_rep = 8 decode attention at full size
+    LLAMA13B.with_(name="llama13b-decode", B=32, T=1, cache_len=4096, decode_steps=2),
+    LLAMA70B.with_(name="llama70b-gqa-decode", B=32, T=1, cache_len=4096, decode_steps=2),
+]
+
+
+@pytest.mark.parametrize("cfg,int8", [(c, False) for c in DECODE_CFGS] + [(DECODE7B, True)],
+                         ids=lambda v: v.name if hasattr(v, "name") else ("int8" if v else "bf16"))
+def test_full_size_decode_step(cfg, int8):
+    """Two decode steps; with int8, the INT8 weight-only path against the oracle run on
+    the dequantized weights."""
+    t_max = cfg.cache_len + 2
     W = make_weights(cfg)
     k0, v0 = make_cache(cfg, t_max)
     blk = lb.LlamaBlock(cfg.d, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.f, cfg.eps, cfg.rope_base,
                         torch.bfloat16, max_pos=t_max)
     blk.set_weights(weights_to_cuda(W))
+    if int8:
+        blk.quantize_decode_weights()
+        W = ob.int8_decode_weights(W)
     kc, vc = k0.cuda(), v0.cuda()
+    del k0, v0
     lens = torch.full((cfg.B,), cfg.cache_len, dtype=torch.int32, device="cuda")
     blk.set_lengths([cfg.cache_len] * cfg.B)
     seqs = [0, 9, 22, 31]
     L = cfg.cache_len
-    kr = as_np(k0[seqs, :, :L + 2])
-    vr = as_np(v0[seqs, :, :L + 2])
+    kr = as_np(kc[seqs, :, :L + 2].cpu())
+    vr = as_np(vc[seqs, :, :L + 2].cpu())
     for s in range(2):
         x = make_decode_x(cfg, s)
         y = torch.empty(cfg.B, 1, cfg.d, dtype=torch.bfloat16, device="cuda")
@@ -78,7 +94,8 @@ def test_full_size_decode_step():
         e_k = row_err(kc[seqs, :, L + s:L + s + 1], want["k_new"])
         e_v = row_err(vc[seqs, :, L + s:L + s + 1], want["v_new"])
         e_b = branch_err(y[seqs], want["y"], want["x1"], want["attn"] + want["mlp"])
-        print(f"decode step {s}: y {e_y:.2e}  k {e_k:.2e}  v {e_v:.2e}  branch {e_b:.2e}")
+        print(f"{cfg.name} {'int8' if int8 else 'bf16'} step {s}: y {e_y:.2e}  k {e_k:.2e}  "
+              f"v {e_v:.2e}  branch {e_b:.2e}")
         assert e_y <= BF16_TOL and e_k <= BF16_TOL and e_v <= BF16_TOL and e_b <= BF16_TOL
         kr[:, :, L + s:L + s + 1], vr[:, :, L + s:L + s + 1] = want["k_new"], want["v_new"]
         assert lens.tolist() == [L + s + 1] * cfg.B

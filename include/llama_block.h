@@ -59,7 +59,10 @@ typedef struct llama_block llama_block; /* opaque, library-owned */
  * num_key_value_heads, head_dim, intermediate_size f; RMSNorm eps §2.1; RoPE base
  * §2.2). `max_pos` sizes the RoPE cos/sin table (positions 0 .. max_pos-1), which
  * the library builds in fp64 on the host. Allocates library-owned device memory
- * (packed weights, RoPE table, error word) on the current device.
+ * (packed weights, RoPE table, error word) on the current device; every later call on
+ * the handle (and on a llama_stack) runs on that device whatever device is current,
+ * and leaves the caller's current device as it was. Its buffers and stream arguments
+ * must belong to that device.
  * Returns LB_ERR_INVALID_ARG for non-positive sizes or a null `out`,
  * LB_ERR_UNSUPPORTED for head_dim not in {64,128} or n_heads / n_kv_heads not in
  * {1, 2, 4, 8}. */

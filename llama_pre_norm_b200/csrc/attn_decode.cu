@@ -280,12 +280,9 @@ static cudaError_t run_split(dim3 grid, const void* q, const void* k, const void
                              float scale_log2, int* err, cudaStream_t s) {
   constexpr int smem = dec_smem_bytes<DH>(NREP);
   auto kern = attn_decode_split_kernel<DH, NREP>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if (cudaError_t e = ensure_smem_attr(kern, smem, attr_done); e != cudaSuccess)
+    return e;
   return launch_k(kern, grid, kDecThreads, smem, s, (const bf16*)q, (const bf16*)k, (const bf16*)v,
                   part, H, Hkv, k_stride, n_splits, kv_len, scale_log2, err);
 }

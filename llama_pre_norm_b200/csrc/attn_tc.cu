@@ -336,12 +336,9 @@ static cudaError_t run_attn(const void* q, const void* k, const void* v, void* o
       !make_tmap_3d_bf16(&tv, v, (uint64_t)B * Hkv, Tk, DH, (uint64_t)k_stride * DH, 128))
     return cudaErrorInvalidValue;
   auto kern = attn_tc_kernel<DH>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if (cudaError_t e = ensure_smem_attr(kern, C::SMEM, attr_done); e != cudaSuccess)
+    return e;
   const int npairs = (Tq + 255) / 256;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
   return launch_k(kern, npairs * B * H, kAttnTcThreads, C::SMEM, s, tq, tk, tv, (bf16*)o, B, Tq, Tk,

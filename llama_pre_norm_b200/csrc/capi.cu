@@ -111,6 +111,28 @@ static int num_sms_of_current_device() {
 }
 
 // Error word of the standalone entry points, one per device.
+// Makes the device a handle was created on current for the duration of a call (the
+// caller's current device may differ), restoring the caller's afterwards.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (dev < 0) return;  // no handle: stay on the current device
+    if (cudaGetDevice(&prev) != cudaSuccess) {
+      prev = -1;
+      ok = false;
+    } else if (prev != dev && cudaSetDevice(dev) != cudaSuccess) {
+      ok = false;
+    }
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+#define LB_ON_DEVICE(h, where)                                                   \
+  DeviceGuard lb_device_guard((h)->device);                                      \
+  if (!lb_device_guard.ok) return fail(LB_ERR_CUDA, "%s: cannot select the handle's device", where)
+
 static std::mutex g_err_mu;
 static std::map<int, int*> g_err_words;
 
@@ -406,6 +428,7 @@ lb_status llama_block_create(int d, int n_heads, int n_kv_heads, int head_dim, i
 
 void llama_block_destroy(llama_block* b) {
   if (!b) return;
+  DeviceGuard dg(b->device);
   cudaDeviceSynchronize();
   for (cudaEvent_t e : b->ev) cudaEventDestroy(e);
   for (void* p : {b->w_qkv, b->w_o, b->w_gu, b->w_d, b->g1, b->g2, (void*)b->cos_t,
@@ -445,6 +468,7 @@ lb_status llama_block_set_weights(llama_block* b, const void* wq, const void* wk
                                   const void* w_down, const void* g_attn, const void* g_mlp,
                                   void* stream) {
   if (!b) return fail(LB_ERR_INVALID_ARG, "set_weights: NULL handle");
+  LB_ON_DEVICE(b, "set_weights");
   if (!wq || !wk || !wv || !wo || !w_gate || !w_up || !w_down || !g_attn || !g_mlp)
     return fail(LB_ERR_INVALID_ARG, "set_weights: NULL weight pointer");
   cudaStream_t s = (cudaStream_t)stream;
@@ -497,6 +521,7 @@ lb_status llama_block_set_weights(llama_block* b, const void* wq, const void* wk
 
 lb_status llama_block_quantize_decode_weights(llama_block* b, int enable, void* stream) {
   if (!b) return fail(LB_ERR_INVALID_ARG, "quantize_decode_weights: NULL handle");
+  LB_ON_DEVICE(b, "quantize_decode_weights");
   if (!enable) {
     LB_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
     for (int i = 0; i < 4; ++i) {
@@ -523,6 +548,7 @@ lb_status llama_block_quantize_decode_weights(llama_block* b, int enable, void* 
 
 lb_status llama_block_reserve(llama_block* b, int max_tokens, int max_batch) {
   if (!b) return fail(LB_ERR_INVALID_ARG, "reserve: NULL handle");
+  LB_ON_DEVICE(b, "reserve");
   if (max_tokens < 0 || max_batch < 0) return fail(LB_ERR_INVALID_ARG, "reserve: negative size");
   size_t a = 0, c = 0;
   carve_prefill(b, nullptr, max_tokens, &a);
@@ -616,6 +642,7 @@ lb_status llama_block_prefill(llama_block* b, const void* x, void* y, int B, int
                               void* v_cache, int t_max, int32_t* cache_len, void* stream) {
   lb_status st = check_cache_args(b, x, y, B, k_cache, v_cache, t_max, cache_len, "prefill");
   if (st != LB_OK) return st;
+  LB_ON_DEVICE(b, "prefill");
   if (T <= 0) return fail(LB_ERR_INVALID_ARG, "prefill: T must be positive");
   if (T > t_max || T > b->max_pos)
     return fail(LB_ERR_CACHE_FULL, "prefill: T=%d exceeds t_max=%d or max_pos=%d", T, t_max,
@@ -627,6 +654,7 @@ lb_status llama_block_extend(llama_block* b, const void* x, void* y, int B, int 
                              void* v_cache, int t_max, int32_t* cache_len, void* stream) {
   lb_status st = check_cache_args(b, x, y, B, k_cache, v_cache, t_max, cache_len, "extend");
   if (st != LB_OK) return st;
+  LB_ON_DEVICE(b, "extend");
   if (T <= 0) return fail(LB_ERR_INVALID_ARG, "extend: T must be positive");
   if ((int)b->lens.size() != B)
     return fail(LB_ERR_INVALID_ARG,
@@ -646,6 +674,7 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
                              void* v_cache, int t_max, int32_t* cache_len, void* stream) {
   lb_status st = check_cache_args(b, x, y, B, k_cache, v_cache, t_max, cache_len, "decode");
   if (st != LB_OK) return st;
+  LB_ON_DEVICE(b, "decode");
   if ((int)b->lens.size() != B)
     return fail(LB_ERR_INVALID_ARG,
                 "decode: the handle knows %d sequence lengths, B=%d (call prefill or set_lengths)",
@@ -738,6 +767,7 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
 
 lb_status llama_block_enable_timing(llama_block* b, int enable) {
   if (!b) return fail(LB_ERR_INVALID_ARG, "enable_timing: NULL handle");
+  LB_ON_DEVICE(b, "enable_timing");
   if (enable && b->ev.empty()) {
     b->ev.resize(2 * kMaxStages);
     for (auto& e : b->ev) LB_CUDA(cudaEventCreate(&e));
@@ -749,6 +779,7 @@ lb_status llama_block_enable_timing(llama_block* b, int enable) {
 lb_status llama_block_stage_times(llama_block* b, float* ms, int max_stages, int* n_stages) {
   if (!b || !n_stages) return fail(LB_ERR_INVALID_ARG, "stage_times: NULL argument");
   if (!b->timing) return fail(LB_ERR_INVALID_ARG, "stage_times: timing is not enabled");
+  LB_ON_DEVICE(b, "stage_times");
   const int n = std::min((int)b->stage_names.size(), kMaxStages);
   *n_stages = n;
   for (int i = 0; i < n && i < max_stages && ms; ++i) {
@@ -771,6 +802,8 @@ static const char* describe_err(int code) {
 }
 
 lb_status llama_block_sync_status(llama_block* b, void* stream) {
+  DeviceGuard dg(b ? b->device : -1);
+  if (b && !dg.ok) return fail(LB_ERR_CUDA, "sync_status: cannot select the handle's device");
   int* word = b ? b->err : standalone_err_word();
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return fail(LB_ERR_CUDA, "sync_status: %s", cudaGetErrorString(e));
@@ -912,6 +945,7 @@ lb_status swiglu_mlp(const void* h, const void* w_gate, const void* w_up, const 
 // owns two ping-pong activation buffers and one device length array per layer.
 struct llama_stack {
   std::vector<llama_block*> layers;
+  int device = 0;  // the device of every layer (current at creation)
   int d = 0;
   size_t esz = 0;
   void* act[2] = {nullptr, nullptr};
@@ -924,6 +958,7 @@ extern "C" {
 
 void llama_stack_destroy(llama_stack* st) {
   if (!st) return;
+  DeviceGuard dg(st->device);
   cudaDeviceSynchronize();
   for (llama_block* b : st->layers) llama_block_destroy(b);
   for (void* p : {st->act[0], st->act[1], (void*)st->lens})
@@ -938,6 +973,10 @@ lb_status llama_stack_create(int n_layers, int d, int n_heads, int n_kv_heads, i
   *out = nullptr;
   if (n_layers <= 0) return fail(LB_ERR_INVALID_ARG, "stack_create: n_layers must be positive");
   llama_stack* st = new llama_stack();
+  if (cudaGetDevice(&st->device) != cudaSuccess) {
+    delete st;
+    return fail(LB_ERR_CUDA, "stack_create: no CUDA device");
+  }
   for (int l = 0; l < n_layers; ++l) {
     llama_block* b = nullptr;
     const lb_status r =
@@ -981,6 +1020,7 @@ static lb_status stack_run(llama_stack* st, StackOp op, const void* x, void* y, 
     return fail(LB_ERR_INVALID_ARG, "%s: NULL argument", who);
   if (B <= 0 || T <= 0) return fail(LB_ERR_INVALID_ARG, "%s: B and T must be positive", who);
   if (x == y) return fail(LB_ERR_INVALID_ARG, "%s: y must not alias x", who);
+  LB_ON_DEVICE(st, who);
   const int n = (int)st->layers.size();
   for (int l = 0; l < n; ++l)
     if (!k_caches[l] || !v_caches[l])

@@ -623,12 +623,9 @@ static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int M, int 
                        int kb_per, int n_split, const GemmEpi& epi, int grid, cudaStream_t s) {
   using C = GemmCfg<BN>;
   auto kern = gemm_tc_kernel<BN, EPI>;
-  static bool attr_set = false;  // per instantiation; the attribute is per device function
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if (cudaError_t e = ensure_smem_attr(kern, C::SMEM, attr_done); e != cudaSuccess)
+    return e;
   return launch_k(kern, grid, kGemmThreads, C::SMEM, s, ta, tb, M, N, K, kb_per, n_split, epi);
 }
 
@@ -637,12 +634,9 @@ static cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int M,
                             const GemmEpi& epi, int grid, cudaStream_t s) {
   using C = Gemm2Cfg<BN>;
   auto kern = gemm_tc_pair_kernel<BN, EPI>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if (cudaError_t e = ensure_smem_attr(kern, C::SMEM, attr_done); e != cudaSuccess)
+    return e;
   return launch_k_pair(kern, grid, kGemmThreads, C::SMEM, s, ta, tb, M, N, K, epi);
 }
 

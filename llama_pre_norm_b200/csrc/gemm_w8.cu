@@ -360,12 +360,9 @@ cudaError_t launch_gemm_w8(const void* A8, const float* row_scale, const void* B
   const long long units = (long long)((M + 127) / 128) * n_split;
   const int grid = (int)std::min<long long>(units, num_sms);
   auto kern = gemm_w8_kernel<BN>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if (cudaError_t e = ensure_smem_attr(kern, C::SMEM, attr_done); e != cudaSuccess)
+    return e;
   return launch_k(kern, grid, kW8Threads, C::SMEM, s, (const uint8_t*)A8, tb, row_scale, M, N, K,
                   kt_per, n_split, epi);
 }

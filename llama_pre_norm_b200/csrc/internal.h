@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
 
 namespace lb {
 
@@ -26,6 +27,21 @@ inline int gemm_effective_split(int K, int n_split) {
   n_split = std::max(1, std::min(n_split, KB));
   const int per = (KB + n_split - 1) / n_split;
   return (KB + per - 1) / per;
+}
+
+// Raise `kern`'s dynamic shared-memory limit to `bytes` once per device: the attribute
+// is per device and a process may drive several GPUs. `done` (one static per kernel)
+// holds a bit per device ordinal < 64; larger ordinals set the attribute every time.
+template <typename Kern>
+inline cudaError_t ensure_smem_attr(Kern kern, int bytes, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
 }
 
 // Launch `kern` on `s` with programmatic dependent launch allowed: the grid may

@@ -162,3 +162,15 @@ def test_cache_full_and_missing_lengths_are_rejected_on_host():
         fresh.prefill(cuda(make_x(cfg)), torch.empty(1, 8, cfg.d, device="cuda"), kc, vc, lens)
     assert ei.value.name == "LB_ERR_NO_WEIGHTS"
     fresh.close()
+
+
+def test_calls_leave_the_current_device_unchanged():
+    """Handle calls select the handle's device for their duration and restore the
+    caller's (with one GPU both are device 0; the call must not disturb it)."""
+    cfg = TINY_F32.with_(B=1, T=8)
+    before = torch.cuda.current_device()
+    blk, y, kc, vc, lens = _run_prefill(cfg, make_x(cfg), make_weights(cfg), t_max=16)
+    blk.sync_status()
+    assert torch.cuda.current_device() == before
+    blk.close()
+    assert torch.cuda.current_device() == before

@@ -391,6 +391,11 @@ class LlamaStack:
         llama_block_set_weights(h, w["wq"], w["wk"], w["wv"], w["wo"], w["w_gate"], w["w_up"],
                                 w["w_down"], w["g_attn"], w["g_mlp"], stream)
 
+    def quantize_decode_weights(self, enable=True, stream=None):
+        """INT8 weight-only decode projections for every layer (or back to bf16)."""
+        for layer in range(self.n_layers):
+            llama_block_quantize_decode_weights(llama_stack_layer(self.handle, layer), enable, stream)
+
     def prefill(self, x, y, k_caches, v_caches, cache_len, stream=None):
         llama_stack_prefill(self.handle, x, y, k_caches, v_caches, cache_len, stream)
 

@@ -150,3 +150,48 @@ def test_stack_prefill_extend_decode(dtype):
         L += 1
         assert lens.tolist() == [L] * cfg.B
     st.close()
+
+
+def test_stack_decode_with_int8_weights():
+    """INT8 weight-only decode through a 3-layer stack: every layer against the oracle
+    run on its dequantized INT8 weights."""
+    n_layers = 3
+    cfg = BlockConfig("stack-int8", d=256, n_heads=4, n_kv_heads=2, head_dim=128, f=512, B=2, T=1,
+                      dtype="bf16")
+    Ws = [make_weights(cfg, seed=20 + l) for l in range(n_layers)]
+    T1 = 70
+    X = make_x(cfg, T=T1)
+    t_max = T1 + 4
+    st = lb.LlamaStack(n_layers, cfg.d, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.f, cfg.eps,
+                       cfg.rope_base, torch.bfloat16, max_pos=t_max)
+    for l in range(n_layers):
+        st.set_layer_weights(l, weights_to_cuda(Ws[l]))
+    kcs = [torch.zeros(cfg.B, cfg.n_kv_heads, t_max, cfg.head_dim, dtype=torch.bfloat16, device="cuda")
+           for _ in range(n_layers)]
+    vcs = [torch.zeros_like(k) for k in kcs]
+    lens = torch.zeros(cfg.B, dtype=torch.int32, device="cuda")
+    y1 = torch.empty(cfg.B, T1, cfg.d, dtype=torch.bfloat16, device="cuda")
+    st.prefill(cuda(X), y1, kcs, vcs, lens)  # prefill keeps the bf16 weights
+    st.quantize_decode_weights()
+    torch.cuda.synchronize()
+    ref = ob.stack_prefill(X, Ws, *_oracle_args(cfg))
+    W8s = [ob.int8_decode_weights(W) for W in Ws]
+    kr = [np.concatenate([ref["k"][l], np.zeros((cfg.B, cfg.n_kv_heads, 4, cfg.head_dim))], axis=2)
+          for l in range(n_layers)]
+    vr = [np.concatenate([ref["v"][l], np.zeros((cfg.B, cfg.n_kv_heads, 4, cfg.head_dim))], axis=2)
+          for l in range(n_layers)]
+    L = T1
+    for s in range(2):
+        x = make_decode_x(cfg, s)
+        yd = torch.empty(cfg.B, 1, cfg.d, dtype=torch.bfloat16, device="cuda")
+        st.decode(cuda(x), yd, kcs, vcs, lens)
+        lb.llama_block_sync_status()
+        torch.cuda.synchronize()
+        h = x
+        for l in range(n_layers):
+            out = ob.block_decode(h, W8s[l], *_oracle_args(cfg), kr[l], vr[l], [L] * cfg.B)
+            kr[l][:, :, L:L + 1], vr[l][:, :, L:L + 1] = out["k_new"], out["v_new"]
+            h = out["y"]
+        assert row_err(yd, h) <= BF16_TOL
+        L += 1
+    st.close()

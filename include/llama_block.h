@@ -213,7 +213,48 @@ lb_status llama_stack_set_lengths(llama_stack* st, const int32_t* lens_host, int
 /* Free the stack, its layers and its buffers. */
 void llama_stack_destroy(llama_stack* st);
 
+/* ---------------- tensor parallelism ---------------- */
+
+/* "深入解析Llama MLP模块" page §6.3: the block split over W ranks, Megatron style: rank r
+ * holds query heads [r H/W, (r+1) H/W), KV heads [r H_kv/W, ..), intermediate columns
+ * [r f/W, ..); Q/K/V and gate/up are split by output rows, o_proj and down by input
+ * columns, and an all-reduce over ranks completes each branch. A shard is an ordinary
+ * handle created with (d, H/W, H_kv/W, head_dim, f/W) and given its weight slices (the
+ * RMSNorm gains whole); its KV cache holds its KV heads. bf16 handles only
+ * (LB_ERR_UNSUPPORTED otherwise); LB_ERR_NO_WEIGHTS before set_weights. One layer:
+ *   tp_attn_*(x) -> o_part     all-reduce(o_part) -> o_sum
+ *   tp_mlp(x, o_sum) -> x1, m_part     all-reduce(m_part) -> m_sum
+ *   tp_add(x1, m_sum) -> y     (y = x + o + m, the block output)
+ * The all-reduce is the caller's (e.g. NCCL). Partials are bf16 [rows, d]. */
+
+/* Attention branch of a fresh prefill (T tokens per sequence at positions 0..T-1): the
+ * rank's Q/K/V with RoPE (its K/V written to cache positions [0, T)), causal attention of
+ * its heads, and o_part [B, T, d] = O_rank W_o[:, rank]^T (no residual). Sets cache_len
+ * and the handle's lengths to T. Errors as llama_block_prefill. */
+lb_status llama_block_tp_attn_prefill(llama_block* shard, const void* x, void* o_part, int B, int T,
+                                      void* k_cache, void* v_cache, int t_max, int32_t* cache_len,
+                                      void* stream);
+
+/* Attention branch of one decode step (one token per sequence at position cache_len[b],
+ * its K/V appended there): o_part [B, 1, d] as above; cache_len += 1. Uses the INT8
+ * weights when they are enabled. Errors as llama_block_decode. */
+lb_status llama_block_tp_attn_decode(llama_block* shard, const void* x, void* o_part, int B,
+                                     void* k_cache, void* v_cache, int t_max, int32_t* cache_len,
+                                     void* stream);
+
+/* MLP branch for M token rows: x1 = x + o_sum (written, [M, d]), then m_part [M, d] =
+ * (SiLU(RMSNorm(x1) W_gate[rank]^T) * RMSNorm(x1) W_up[rank]^T) W_down[:, rank]^T. x1
+ * and m_part must not alias the inputs (LB_ERR_INVALID_ARG). */
+lb_status llama_block_tp_mlp(llama_block* shard, const void* x, const void* o_sum, void* x1,
+                             void* m_part, int M, void* stream);
+
+/* out = a + b, rows x d elements of `dtype` (d % 8 == 0), fp32 add with one rounding: the
+ * residual stream plus an all-reduced branch. */
+lb_status llama_block_tp_add(const void* a, const void* b, void* out, int rows, int d, lb_dtype dtype,
+                             void* stream);
+
 /* ---------------- standalone entry points (testing) ---------------- */
+
 
 /* RMSNorm (LMDrive page §2.1; mechanics page §02.3): y = g * x / sqrt(mean(x^2) + eps)
  * over the last axis, fp32 accumulation, one rounding. x, y: [rows, d]; g: [d].

@@ -27,6 +27,8 @@ __all__ = [
     "rmsnorm", "rope_apply", "causal_attn", "swiglu_mlp", "decode_attn_static_scratch", "LlamaBlock",
     "llama_stack_create", "llama_stack_layer", "llama_stack_prefill", "llama_stack_extend",
     "llama_stack_decode", "llama_stack_set_lengths", "llama_stack_destroy", "LlamaStack",
+    "llama_block_tp_attn_prefill", "llama_block_tp_attn_decode", "llama_block_tp_mlp",
+    "llama_block_tp_add", "tp_shard_weights",
 ]
 
 LB_F32, LB_BF16 = 0, 1
@@ -47,6 +49,10 @@ _SIGS = {
     "llama_block_set_weights": (_i, [_p] * 11),
     "llama_block_reserve": (_i, [_p, _i, _i]),
     "llama_block_quantize_decode_weights": (_i, [_p, _i, _p]),
+    "llama_block_tp_attn_prefill": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p]),
+    "llama_block_tp_attn_decode": (_i, [_p, _p, _p, _i, _p, _p, _i, _p, _p]),
+    "llama_block_tp_mlp": (_i, [_p, _p, _p, _p, _p, _i, _p]),
+    "llama_block_tp_add": (_i, [_p, _p, _p, _i, _i, _i, _p]),
     "llama_block_prefill": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p]),
     "llama_block_extend": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p]),
     "llama_block_decode": (_i, [_p, _p, _p, _i, _p, _p, _i, _p, _p]),
@@ -171,6 +177,62 @@ def llama_block_decode(h, x, y, k_cache, v_cache, cache_len, stream=None):
                                   _ptr(k_cache, "k_cache", x.dtype), _ptr(v_cache, "v_cache", x.dtype),
                                   t_max, _ptr(cache_len, "cache_len", torch.int32), _stream(stream)),
            "llama_block_decode")
+
+
+# ----------------------------------------------------------------- tensor parallelism
+def tp_shard_weights(W: dict, rank: int, world: int, n_heads: int, n_kv_heads: int,
+                     head_dim: int) -> dict:
+    """Rank `rank`'s slice of a block's nn.Linear weights ("深入解析Llama MLP模块" page
+    §6.3, Megatron split): q/k/v rows of its heads and gate/up rows of its intermediate
+    columns (column-parallel), o_proj and down columns of the same (row-parallel); the
+    RMSNorm gains whole. Argument slicing only; the shard handle is created with
+    (d, n_heads // world, n_kv_heads // world, head_dim, f // world)."""
+    f = W["w_gate"].shape[0]
+    if n_heads % world or n_kv_heads % world or f % world:
+        raise ValueError("n_heads, n_kv_heads and f must divide by the number of ranks")
+    hq, hk, fs = n_heads // world, n_kv_heads // world, f // world
+    q0, k0, f0 = rank * hq * head_dim, rank * hk * head_dim, rank * fs
+    return {
+        "wq": W["wq"][q0:q0 + hq * head_dim].contiguous(),
+        "wk": W["wk"][k0:k0 + hk * head_dim].contiguous(),
+        "wv": W["wv"][k0:k0 + hk * head_dim].contiguous(),
+        "wo": W["wo"][:, q0:q0 + hq * head_dim].contiguous(),
+        "w_gate": W["w_gate"][f0:f0 + fs].contiguous(),
+        "w_up": W["w_up"][f0:f0 + fs].contiguous(),
+        "w_down": W["w_down"][:, f0:f0 + fs].contiguous(),
+        "g_attn": W["g_attn"], "g_mlp": W["g_mlp"],
+    }
+
+
+def llama_block_tp_attn_prefill(h, x, o_part, k_cache, v_cache, cache_len, stream=None):
+    B, T, _ = x.shape
+    _check(lib.llama_block_tp_attn_prefill(h, _ptr(x, "x"), _ptr(o_part, "o_part", x.dtype), B, T,
+                                           _ptr(k_cache, "k_cache", x.dtype),
+                                           _ptr(v_cache, "v_cache", x.dtype), k_cache.shape[2],
+                                           _ptr(cache_len, "cache_len", torch.int32), _stream(stream)),
+           "llama_block_tp_attn_prefill")
+
+
+def llama_block_tp_attn_decode(h, x, o_part, k_cache, v_cache, cache_len, stream=None):
+    _check(lib.llama_block_tp_attn_decode(h, _ptr(x, "x"), _ptr(o_part, "o_part", x.dtype), x.shape[0],
+                                          _ptr(k_cache, "k_cache", x.dtype),
+                                          _ptr(v_cache, "v_cache", x.dtype), k_cache.shape[2],
+                                          _ptr(cache_len, "cache_len", torch.int32), _stream(stream)),
+           "llama_block_tp_attn_decode")
+
+
+def llama_block_tp_mlp(h, x, o_sum, x1, m_part, stream=None):
+    M = x.numel() // x.shape[-1]
+    _check(lib.llama_block_tp_mlp(h, _ptr(x, "x"), _ptr(o_sum, "o_sum", x.dtype), _ptr(x1, "x1", x.dtype),
+                                  _ptr(m_part, "m_part", x.dtype), M, _stream(stream)),
+           "llama_block_tp_mlp")
+
+
+def llama_block_tp_add(a, b, out, stream=None):
+    d = a.shape[-1]
+    _check(lib.llama_block_tp_add(_ptr(a, "a"), _ptr(b, "b", a.dtype), _ptr(out, "out", a.dtype),
+                                  a.numel() // d, d, dtype_code(a.dtype), _stream(stream)),
+           "llama_block_tp_add")
 
 
 def llama_block_set_lengths(h, lens):

@@ -765,6 +765,164 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
   return LB_OK;
 }
 
+// ---------------------------------------------------------------- tensor parallelism
+// "深入解析Llama MLP模块" page §6.3: with the block split over ranks (Q/K/V and gate/up
+// split by output rows, o_proj and down by input columns), each rank computes a partial
+// sum of the attention branch and of the MLP branch, and an all-reduce over ranks
+// completes each. A shard handle is an ordinary handle created with the rank's head
+// counts and intermediate size and given the rank's weight slices; these calls run its
+// partial branches. bf16 handles only.
+static lb_status tp_check(llama_block* b, const char* who) {
+  if (!b) return fail(LB_ERR_INVALID_ARG, "%s: NULL handle", who);
+  if (b->dtype != kBF16) return fail(LB_ERR_UNSUPPORTED, "%s: tensor-parallel shards need LB_BF16", who);
+  if (!b->has_weights) return fail(LB_ERR_NO_WEIGHTS, "%s: set_weights first", who);
+  return LB_OK;
+}
+
+lb_status llama_block_tp_attn_prefill(llama_block* b, const void* x, void* o_part, int B, int T,
+                                      void* k_cache, void* v_cache, int t_max, int32_t* cache_len,
+                                      void* stream) {
+  lb_status st = check_cache_args(b, x, o_part, B, k_cache, v_cache, t_max, cache_len, "tp_attn_prefill");
+  if (st != LB_OK) return st;
+  if ((st = tp_check(b, "tp_attn_prefill")) != LB_OK) return st;
+  LB_ON_DEVICE(b, "tp_attn_prefill");
+  if (T <= 0) return fail(LB_ERR_INVALID_ARG, "tp_attn_prefill: T must be positive");
+  if (T > t_max || T > b->max_pos)
+    return fail(LB_ERR_CACHE_FULL, "tp_attn_prefill: T=%d exceeds t_max=%d or max_pos=%d", T, t_max,
+                b->max_pos);
+  cudaStream_t s = (cudaStream_t)stream;
+  const int M = B * T;
+  size_t need = 0;
+  carve_prefill(b, nullptr, M, &need);
+  if ((st = ensure_ws(b, need)) != LB_OK) return st;
+  PrefillWs w = carve_prefill(b, b->ws, M, &need);
+  const int d = b->d, H = b->H, Hkv = b->Hkv, dh = b->dh;
+  b->stage_names.clear();
+  LB_STAGE("row_stats_attn", 1, launch_row_ssq(x, w.ss1, w.ss2, M, d, cache_len, B, T, s));
+  GemmEpi e1;
+  e1.kind = kEpiQkvRope;
+  e1.T = T; e1.H = H; e1.Hkv = Hkv; e1.dh = dh; e1.t_max = t_max; e1.max_pos = b->max_pos;
+  e1.q_out = w.q; e1.k_cache = k_cache; e1.v_cache = v_cache; e1.pos0 = 0;
+  e1.cos_t = b->cos_t; e1.sin_t = b->sin_t; e1.err = b->err;
+  e1.row_ss = w.ss1; e1.row_inv_d = 1.f / d; e1.row_eps = b->eps;
+  LB_STAGE("qkv_rope_gemm", 1, launch_gemm_tc(x, b->w_qkv, M, b->n_qkv, d, 256, 1, e1, b->num_sms, s));
+  LB_STAGE("attention", 1, launch_attn_tc(w.q, k_cache, v_cache, w.o, B, T, T, H, Hkv, dh, t_max, b->err, s));
+  GemmEpi e2;  // this shard's o_proj columns: a partial sum, no residual
+  e2.kind = kEpiStore; e2.out = o_part; e2.ldo = d; e2.err = b->err;
+  LB_STAGE("o_proj_partial_gemm", 1, launch_gemm_tc(w.o, b->w_o, M, d, H * dh, 256, 1, e2, b->num_sms, s));
+  b->lens.assign(B, T);
+  return LB_OK;
+}
+
+lb_status llama_block_tp_attn_decode(llama_block* b, const void* x, void* o_part, int B, void* k_cache,
+                                     void* v_cache, int t_max, int32_t* cache_len, void* stream) {
+  lb_status st = check_cache_args(b, x, o_part, B, k_cache, v_cache, t_max, cache_len, "tp_attn_decode");
+  if (st != LB_OK) return st;
+  if ((st = tp_check(b, "tp_attn_decode")) != LB_OK) return st;
+  LB_ON_DEVICE(b, "tp_attn_decode");
+  if ((int)b->lens.size() != B)
+    return fail(LB_ERR_INVALID_ARG, "tp_attn_decode: the handle knows %d sequence lengths, B=%d",
+                (int)b->lens.size(), B);
+  for (int i = 0; i < B; ++i)
+    if (b->lens[i] < 0 || b->lens[i] + 1 > t_max || b->lens[i] >= b->max_pos)
+      return fail(LB_ERR_CACHE_FULL, "tp_attn_decode: sequence %d at length %d cannot grow", i, b->lens[i]);
+  cudaStream_t s = (cudaStream_t)stream;
+  size_t need = 0;
+  carve_decode(b, nullptr, B, t_max, &need);
+  if ((st = ensure_ws(b, need)) != LB_OK) return st;
+  DecodeWs w = carve_decode(b, b->ws, B, t_max, &need);
+  const int d = b->d, H = b->H, Hkv = b->Hkv, dh = b->dh;
+  const DecodePlan plan = decode_plan(b, B, b->decode_int8);
+  auto wgemm = [&](int i, const void* wbf, const void* act, int Mw, int Kw, int split,
+                   const GemmEpi& ep) -> cudaError_t {
+    if (plan.w8) return launch_gemm_w8(b->q8[i], b->s8[i], act, Mw, B, Kw, split, ep, b->num_sms, s);
+    return launch_gemm_tc(wbf, act, Mw, B, Kw, plan.bn, split, ep, b->num_sms, s);
+  };
+  b->stage_names.clear();
+  LB_STAGE("rmsnorm_attn", 1,
+           launch_resid_rmsnorm(kBF16, x, nullptr, 0, 0, nullptr, nullptr, w.h, B, d, b->eps, s));
+  GemmEpi e;
+  e.kind = kEpiPartialT; e.out = w.part; e.err = b->err;
+  e.ldo = b->n_qkv; e.split_stride = (long long)B * b->n_qkv;
+  LB_STAGE("qkv_gemm", 1, wgemm(0, b->w_qkv, w.h, b->n_qkv, d, plan.split[0], e));
+  LB_STAGE("qkv_rope_append", 1,
+           launch_qkv_finish(kBF16, w.part, plan.split[0], e.split_stride, B, 1, H, Hkv, dh, cache_len, 0,
+                             b->cos_t, b->sin_t, b->max_pos, w.q, k_cache, v_cache, t_max, b->err, s));
+  LB_STAGE("attention", 2, launch_attn_decode(w.q, k_cache, v_cache, w.o, w.attn_part, B, H, Hkv, dh, t_max,
+                                              cache_len, b->err, s));
+  e.ldo = d; e.split_stride = (long long)B * d;
+  LB_STAGE("o_proj_gemm", 1, wgemm(1, b->w_o, w.o, d, H * dh, plan.split[1], e));
+  // the partial sum of this shard's o_proj columns; cache_len += 1
+  LB_STAGE("o_partial_len", 1, launch_resid_add(kBF16, nullptr, w.part, plan.split[1], e.split_stride,
+                                                o_part, (long long)B * d, cache_len, B, 1, s));
+  for (int i = 0; i < B; ++i) b->lens[i] += 1;
+  return LB_OK;
+}
+
+lb_status llama_block_tp_mlp(llama_block* b, const void* x, const void* o_sum, void* x1, void* m_part,
+                             int M, void* stream) {
+  lb_status st = tp_check(b, "tp_mlp");
+  if (st != LB_OK) return st;
+  if (!x || !o_sum || !x1 || !m_part) return fail(LB_ERR_INVALID_ARG, "tp_mlp: NULL argument");
+  if (M < 0) return fail(LB_ERR_INVALID_ARG, "tp_mlp: negative row count");
+  if (x1 == x || x1 == o_sum || m_part == x1)
+    return fail(LB_ERR_INVALID_ARG, "tp_mlp: x1 and m_part must not alias the inputs");
+  if (M == 0) return LB_OK;
+  LB_ON_DEVICE(b, "tp_mlp");
+  cudaStream_t s = (cudaStream_t)stream;
+  const int d = b->d, f = b->f;
+  b->stage_names.clear();
+  size_t need = 0;
+  if (M <= 256) {  // decode-sized: swap-AB split-K GEMMs
+    carve_decode(b, nullptr, M, 1, &need);
+    if ((st = ensure_ws(b, need)) != LB_OK) return st;
+    DecodeWs w = carve_decode(b, b->ws, M, 1, &need);
+    const DecodePlan plan = decode_plan(b, M, b->decode_int8);
+    auto wgemm = [&](int i, const void* wbf, const void* act, int Mw, int Kw, int split,
+                     const GemmEpi& ep) -> cudaError_t {
+      if (plan.w8) return launch_gemm_w8(b->q8[i], b->s8[i], act, Mw, M, Kw, split, ep, b->num_sms, s);
+      return launch_gemm_tc(wbf, act, Mw, M, Kw, plan.bn, split, ep, b->num_sms, s);
+    };
+    LB_STAGE("resid_add_attn", 1, launch_add_rows(kBF16, x, o_sum, x1, nullptr, M, d, s));
+    LB_STAGE("rmsnorm_mlp", 1,
+             launch_resid_rmsnorm(kBF16, x1, nullptr, 0, 0, nullptr, nullptr, w.h, M, d, b->eps, s));
+    GemmEpi e;
+    e.kind = kEpiPartialT; e.out = w.part; e.err = b->err;
+    e.ldo = b->n_gu; e.split_stride = (long long)M * b->n_gu;
+    LB_STAGE("gate_up_gemm", 1, wgemm(2, b->w_gu, w.h, b->n_gu, d, plan.split[2], e));
+    LB_STAGE("silu_mul", 1, launch_silu_mul(kBF16, w.part, plan.split[2], e.split_stride, M, f, b->n_gu, 128,
+                                            w.a, s));
+    e.ldo = d; e.split_stride = (long long)M * d;
+    LB_STAGE("down_gemm", 1, wgemm(3, b->w_d, w.a, d, f, plan.split[3], e));
+    LB_STAGE("m_partial", 1, launch_resid_add(kBF16, nullptr, w.part, plan.split[3], e.split_stride, m_part,
+                                              (long long)M * d, nullptr, 0, 0, s));
+    return LB_OK;
+  }
+  carve_prefill(b, nullptr, M, &need);
+  if ((st = ensure_ws(b, need)) != LB_OK) return st;
+  PrefillWs w = carve_prefill(b, b->ws, M, &need);
+  // X' = X + (all-reduced attention partial) with its RMSNorm statistic
+  LB_STAGE("resid_add_attn", 1, launch_add_rows(kBF16, x, o_sum, x1, w.ss2, M, d, s));
+  GemmEpi e3;
+  e3.kind = kEpiSwiGLU; e3.out = w.a; e3.ldo = f; e3.f = f; e3.err = b->err;
+  e3.row_ss = w.ss2; e3.row_inv_d = 1.f / d; e3.row_eps = b->eps;
+  LB_STAGE("gate_up_swiglu_gemm", 1, launch_gemm_tc(x1, b->w_gu, M, b->n_gu, d, 256, 1, e3, b->num_sms, s));
+  GemmEpi e4;  // this shard's down columns: a partial sum, no residual
+  e4.kind = kEpiStore; e4.out = m_part; e4.ldo = d; e4.err = b->err;
+  LB_STAGE("down_partial_gemm", 1, launch_gemm_tc(w.a, b->w_d, M, d, f, 256, 1, e4, b->num_sms, s));
+  return LB_OK;
+}
+
+lb_status llama_block_tp_add(const void* a, const void* b_in, void* out, int rows, int d, lb_dtype dtype,
+                             void* stream) {
+  if (rows < 0 || d <= 0 || d % 8) return fail(LB_ERR_INVALID_ARG, "tp_add: bad shape (d %% 8 == 0)");
+  if (rows == 0) return LB_OK;
+  if (!a || !b_in || !out) return fail(LB_ERR_INVALID_ARG, "tp_add: NULL argument");
+  const int dt = dtype == LB_F32 ? kF32 : kBF16;
+  LB_CUDA(launch_add_rows(dt, a, b_in, out, nullptr, rows, d, (cudaStream_t)stream));
+  return LB_OK;
+}
+
 lb_status llama_block_enable_timing(llama_block* b, int enable) {
   if (!b) return fail(LB_ERR_INVALID_ARG, "enable_timing: NULL handle");
   LB_ON_DEVICE(b, "enable_timing");

@@ -96,6 +96,10 @@ cudaError_t launch_qkv_finish(int dtype, const float* qkv, int n_split, long lon
                               void* k_cache, void* v_cache, int t_max, int* err, cudaStream_t s);
 cudaError_t launch_silu_mul(int dtype, const float* gu, int n_split, long long split_stride, int M,
                             int f, int n_packed, int block, void* a, cudaStream_t s);
+// out = a + b per row of d (d % 8 == 0), with each stored row's sum of squares in ss_out
+// when it is not NULL.
+cudaError_t launch_add_rows(int dtype, const void* a, const void* b, void* out, float* ss_out,
+                            int rows, int d, cudaStream_t s);
 cudaError_t launch_resid_add(int dtype, const void* resid, const float* part, int n_split,
                              long long split_stride, void* out, long long total, int* lens, int B,
                              int len_inc, cudaStream_t s);

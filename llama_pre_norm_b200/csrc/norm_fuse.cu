@@ -223,7 +223,7 @@ __global__ void resid_add_kernel(const T* __restrict__ resid, const float* __res
     for (int b = threadIdx.x; b < B; b += blockDim.x) lens[b] += len_inc;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
-    float v = to_f<T>(resid[idx]);
+    float v = resid ? to_f<T>(resid[idx]) : 0.f;  // no residual: the partials' sum alone
     for (int s = 0; s < n_split; ++s) v += part[s * split_stride + idx];
     out[idx] = from_f<T>(v);
   }
@@ -240,6 +240,48 @@ cudaError_t launch_resid_add(int dtype, const void* resid, const float* part, in
                     n_split, split_stride, (float*)out, total, lens, B, len_inc);
   return launch_k(resid_add_kernel<bf16>, blocks, threads, 0, s, (const bf16*)resid, part, n_split,
                   split_stride, (bf16*)out, total, lens, B, len_inc);
+}
+
+// ---------------------------------------------------------------- row add
+// out = a + b row by row (fp32 add, one rounding), and when ss_out != NULL the sum of
+// squares of each stored (rounded) out row, the statistic the next GEMM's fused RMSNorm
+// reads. Tensor parallelism (Llama-MLP page §6.3): the residual stream plus the
+// all-reduced partial sum of a branch.
+template <typename T>
+__global__ void __launch_bounds__(kNormThreads) add_rows_kernel(const T* __restrict__ a,
+                                                                const T* __restrict__ b,
+                                                                T* __restrict__ out,
+                                                                float* __restrict__ ss_out, int d) {
+  __shared__ float red[32];
+  pdl_wait();
+  pdl_trigger();
+  const long long row = blockIdx.x;
+  float ss = 0.f;
+  for (int vi = threadIdx.x; vi < (d >> 3); vi += kNormThreads) {
+    float va[8], vb[8];
+    load8(a + row * d + vi * 8, va);
+    load8(b + row * d + vi * 8, vb);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      va[e] = round_to<T>(va[e] + vb[e]);
+      ss = fmaf(va[e], va[e], ss);
+    }
+    store8(out + row * d + vi * 8, va);
+  }
+  if (ss_out) {
+    ss = block_sum(ss, red);
+    if (threadIdx.x == 0) ss_out[row] = ss;
+  }
+}
+
+cudaError_t launch_add_rows(int dtype, const void* a, const void* b, void* out, float* ss_out,
+                            int rows, int d, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (dtype == kF32)
+    return launch_k(add_rows_kernel<float>, rows, kNormThreads, 0, s, (const float*)a,
+                    (const float*)b, (float*)out, ss_out, d);
+  return launch_k(add_rows_kernel<bf16>, rows, kNormThreads, 0, s, (const bf16*)a, (const bf16*)b,
+                  (bf16*)out, ss_out, d);
 }
 
 // ---------------------------------------------------------------- row statistics

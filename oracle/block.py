@@ -321,6 +321,34 @@ def block_extend(x, W: dict, n_heads: int, n_kv_heads: int, head_dim: int, eps: 
 # and the 32 decoder layers of [LMDrive] §1/§5: layer l's output is layer l+1's
 # input; each layer has its own KV cache.
 # --------------------------------------------------------------------------
+# --------------------------------------------------------------------------
+# Tensor parallelism — [Llama-MLP] §6.3: with Q/K/V and gate/up split by output rows
+# and o_proj and down by input columns, every rank's branch output is a partial sum;
+# an all-reduce over ranks completes the branch. A rank's slice is itself a block
+# with n_heads / W query heads, n_kv_heads / W KV heads and f / W intermediate columns.
+# --------------------------------------------------------------------------
+def tp_attention_partial(X, Ws: dict, n_heads: int, n_kv_heads: int, head_dim: int, eps: float,
+                         rope_base: float) -> dict:
+    """One rank's attention-branch partial of a prefill (its heads' attention times its
+    o_proj columns, no residual) and the K/V of its heads."""
+    out = block_prefill(X, Ws, n_heads, n_kv_heads, head_dim, eps, rope_base)
+    return {"o": out["attn"], "k": out["k"], "v": out["v"]}
+
+
+def tp_attention_partial_decode(x, Ws: dict, n_heads: int, n_kv_heads: int, head_dim: int,
+                                eps: float, rope_base: float, k_cache, v_cache, cache_len) -> dict:
+    """One rank's attention-branch partial of a decode step over its heads' cache."""
+    out = block_decode(x, Ws, n_heads, n_kv_heads, head_dim, eps, rope_base, k_cache, v_cache,
+                       cache_len)
+    return {"o": out["attn"], "k_new": out["k_new"], "v_new": out["v_new"]}
+
+
+def tp_mlp_partial(X1, Ws: dict, eps: float) -> np.ndarray:
+    """One rank's MLP-branch partial: SwiGLU over its intermediate columns of the full
+    RMSNorm(X'), times its down columns."""
+    return swiglu_mlp(rmsnorm(X1, Ws["g_mlp"], eps), Ws["w_gate"], Ws["w_up"], Ws["w_down"])
+
+
 def stack_prefill(X, Ws: list, n_heads: int, n_kv_heads: int, head_dim: int, eps: float,
                   rope_base: float) -> dict:
     """Prefill through len(Ws) layers. Returns y and the per-layer caches."""

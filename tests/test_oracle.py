@@ -445,3 +445,4 @@ def test_int8_row_quantization_properties():
     Wq = ob.int8_decode_weights(W)
     assert set(Wq) == set(W) and np.array_equal(Wq["g_attn"], W["g_attn"])
     assert not np.array_equal(Wq["wq"], W["wq"])
+

@@ -76,13 +76,13 @@ def test_full_size_decode_step(cfg, int8):
         blk.quantize_decode_weights()
         W = ob.int8_decode_weights(W)
     kc, vc = k0.cuda(), v0.cuda()
+    seqs = [0, 9, 22, 31]
+    L = cfg.cache_len
+    kr = as_np(k0[seqs, :, :L + 2])  # the oracle's cache: the synthetic host data
+    vr = as_np(v0[seqs, :, :L + 2])
     del k0, v0
     lens = torch.full((cfg.B,), cfg.cache_len, dtype=torch.int32, device="cuda")
     blk.set_lengths([cfg.cache_len] * cfg.B)
-    seqs = [0, 9, 22, 31]
-    L = cfg.cache_len
-    kr = as_np(kc[seqs, :, :L + 2].cpu())
-    vr = as_np(vc[seqs, :, :L + 2].cpu())
     for s in range(2):
         x = make_decode_x(cfg, s)
         y = torch.empty(cfg.B, 1, cfg.d, dtype=torch.bfloat16, device="cuda")

@@ -11,7 +11,7 @@ import torch
 
 from oracle import block as ob
 from synth import BlockConfig, make_decode_x, make_weights, make_x
-from tests.helpers import BF16_TOL, as_np, cuda, row_err, weights_to_cuda
+from tests.helpers import BF16_TOL, cuda, row_err, weights_to_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -75,8 +75,10 @@ def test_tp_block_matches_the_unsplit_block(int8):
         for blk in shards:
             blk.quantize_decode_weights()
         W = ob.int8_decode_weights(W)
-    kr = np.concatenate([as_np(c[0]) for c in caches], axis=1)
-    vr = np.concatenate([as_np(c[1]) for c in caches], axis=1)
+    # the oracle's own prefill K/V as the decode reference's cache
+    kr = np.zeros((cfg.B, cfg.n_kv_heads, t_max, cfg.head_dim))
+    vr = np.zeros_like(kr)
+    kr[:, :, :cfg.T], vr[:, :, :cfg.T] = ref["k"], ref["v"]
     L = cfg.T
     for s in range(2):
         x = make_decode_x(cfg, s)

@@ -22,7 +22,8 @@
 //                measured 3% slower.)
 //   warps 2..5   softmax of tile A, warps 6..9 softmax of tile B: one query row per
 //                thread (= TMEM lane); online max/sum in fp32 with log2(e)/sqrt(d_h)
-//                folded into the exponent's FMA and a three-input max (measured:
+//                folded into the exponent's FMA and a three-input max over eight
+//                independent chains (measured:
 //                packed f32x2 forms and an FMA-pipe polynomial for part of the
 //                exponentials were slower here). The running max is only
 //                moved (and O rescaled in TMEM) when a row's max grows by more than
@@ -240,12 +241,22 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (j * C::BKV + c * 32 + i > qp) s[c][i] = -INFINITY;
       }
-      // row max of the raw scores (the scale is positive), three at a time
-      float mxr = -INFINITY;
+      // row max of the raw scores (the scale is positive), three at a time in eight
+      // independent chains, so that the exponentials wait for a short tree rather
+      // than for 64 dependent steps
+      float m8[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 4; ++c) {
+        m8[2 * c] = -INFINITY;
+        m8[2 * c + 1] = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) mxr = max3(mxr, s[c][i], s[c][i + 1]);
+        for (int i = 0; i < 32; i += 4) {
+          m8[2 * c] = max3(m8[2 * c], s[c][i], s[c][i + 1]);
+          m8[2 * c + 1] = max3(m8[2 * c + 1], s[c][i + 2], s[c][i + 3]);
+        }
+      }
+      const float mxr =
+          max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
       const float mx = mxr * scale_log2;
       // Move the reference max only when this row's max grew by more than 2^8
       // (always on the first tile, where the reference is still -inf).

@@ -327,7 +327,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();  // inputs of the previous kernel are complete and visible from here on
+  // Inputs of the previous kernel are complete and visible after pdl_wait. The weight
+  // operand (A in the swap-AB decode form, B otherwise) is no such input: the producer
+  // fills the ring with the first weight tiles before it waits.
+  if (warp != 0) pdl_wait();
 
   const int num_m = (M + kBM - 1) / kBM, num_n = (N + BN - 1) / BN;
   const int KB = (K + kBK - 1) / kBK;
@@ -336,19 +339,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer
+      constexpr bool kAIsWeight = EPI == kEpiPartialT;
+      int npre = 0;  // leading k-blocks of the first unit whose weight tile is in flight
+      if ((int)blockIdx.x < units) {
+        const Unit w = decode_unit(blockIdx.x, num_m, num_n, KB, kb_per);
+        npre = min(w.kb1 - w.kb0, C::STAGES);
+        for (int i = 0; i < npre; ++i) {  // fresh ring: stage i is free
+          const int kb = w.kb0 + i;
+          mbar_arrive_expect_tx(&full[i], C::STAGE_BYTES);
+          if (kAIsWeight)
+            tma_load_2d(sA + i * C::A_BYTES, &tmA, &full[i], kb * kBK, w.mt * kBM);
+          else
+            tma_load_2d(sB + i * C::B_BYTES, &tmB, &full[i], kb * kBK, w.nt * BN);
+        }
+      }
+      pdl_wait();
       uint32_t stage = 0, phase = 0;
       long long issued = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const Unit w = decode_unit(u, num_m, num_n, KB, kb_per);
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, epi.err, 1)) {
-            ok = false;
-            break;
+          const bool pre = issued < npre;  // weight tile already requested above
+          if (!pre) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, epi.err, 1)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
           }
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * kBK, w.mt * kBM);
-          tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * kBK, w.nt * BN);
+          if (!pre || !kAIsWeight)
+            tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * kBK, w.mt * kBM);
+          if (!pre || kAIsWeight)
+            tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * kBK, w.nt * BN);
           ++issued;
           if (++stage == C::STAGES) {
             stage = 0;

@@ -146,7 +146,9 @@ __global__ void __launch_bounds__(kW8Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();
+  // The INT8 weight tiles are not an input of the previous kernel: the producer
+  // requests the first ones before it waits for that kernel (pdl_wait).
+  if (warp != 0) pdl_wait();
 
   const int num_m = (M + 127) / 128, num_n = (N + BN - 1) / BN;
   const int KT = (K + kW8K - 1) / kW8K;
@@ -164,6 +166,18 @@ __global__ void __launch_bounds__(kW8Threads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- loads; slot reuse needs both its INT8 tile read and its MMAs done
+      int npre = 0;  // leading steps of the first unit whose INT8 tile is in flight
+      if ((int)blockIdx.x < units) {
+        int mt, nt, sp, kt0, kt1;
+        decode(blockIdx.x, mt, nt, sp, kt0, kt1);
+        npre = min(kt1 - kt0, RS);
+        for (int i = 0; i < npre; ++i) {  // fresh ring: slot i is free
+          mbar_arrive_expect_tx(&full[i], C::RAW_BYTES + C::B_BYTES);
+          bulk_load(sRaw + i * C::RAW_BYTES, A8 + ((long long)mt * KT + kt0 + i) * C::RAW_BYTES,
+                    C::RAW_BYTES, &full[i]);
+        }
+      }
+      pdl_wait();
       uint32_t stage = 0, phase = 0;
       long long issued = 0;
       bool ok = true;
@@ -171,15 +185,17 @@ __global__ void __launch_bounds__(kW8Threads, 1)
         int mt, nt, sp, kt0, kt1;
         decode(u, mt, nt, sp, kt0, kt1);
         for (int kt = kt0; kt < kt1; ++kt) {
-          if (!mbar_wait(&raw_free[stage], phase ^ 1, epi.err, 0x41) ||
-              !mbar_wait(&mma_done[stage], phase ^ 1, epi.err, 0x4a)) {
-            ok = false;
-            break;
+          if (issued >= npre) {
+            if (!mbar_wait(&raw_free[stage], phase ^ 1, epi.err, 0x41) ||
+                !mbar_wait(&mma_done[stage], phase ^ 1, epi.err, 0x4a)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[stage], C::RAW_BYTES + C::B_BYTES);
+            // one contiguous tile of the blocked layout
+            bulk_load(sRaw + stage * C::RAW_BYTES, A8 + ((long long)mt * KT + kt) * C::RAW_BYTES,
+                      C::RAW_BYTES, &full[stage]);
           }
-          mbar_arrive_expect_tx(&full[stage], C::RAW_BYTES + C::B_BYTES);
-          // one contiguous tile of the blocked layout
-          bulk_load(sRaw + stage * C::RAW_BYTES, A8 + ((long long)mt * KT + kt) * C::RAW_BYTES,
-                    C::RAW_BYTES, &full[stage]);
           // the token tile in 64-deep pieces (past K they read as zeros)
           uint8_t* b = sB + stage * C::B_BYTES;
 #pragma unroll

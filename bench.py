@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--decode-steps", type=int, default=128)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="also write nvidia-smi clock samples of the timed region to this CSV file")
     return ap.parse_args()
 
 
@@ -134,15 +136,17 @@ def replica_throughput(units_per_rank_step: int, steps: int, world: int, slowest
 class ClockSampler:
     """Samples SM clock, power and clock-event reasons while the timed work runs:
     an NVML thread every 10 ms (read-only queries; the GPU is found by UUID) and,
-    beside it, the nvidia-smi query line of the profiling recipe (200 ms) written
-    to gpurun_out/clocks_gpu<i>.csv."""
+    when a CSV path is given (--clocks-csv), beside it an nvidia-smi query of the
+    same quantities every 200 ms written to that file."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, cuda_index: int):
+    def __init__(self, cuda_index: int, csv_path: str | None = None):
         self.cuda_index = cuda_index
+        self.csv_path = csv_path
+        self.uuid = None
         self.proc = None
         self.samples = []  # (sm_mhz, power_w, reasons bitmask)
         self._stop = None
@@ -169,6 +173,7 @@ class ClockSampler:
             import torch
             nv.nvmlInit()
             uuid = "GPU-" + str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            self.uuid = uuid
             handle = nv.nvmlDeviceGetHandleByUUID(uuid)
             self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
             self._nv = nv
@@ -176,14 +181,17 @@ class ClockSampler:
             self._thread.start()
         except Exception:
             self._thread = None
-        out = ROOT / "gpurun_out"
-        out.mkdir(exist_ok=True)
-        try:
-            self.fh = open(out / f"clocks_gpu{self.cuda_index}.csv", "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv", "-lms", "200"],
-                                         stdout=self.fh, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        if self.csv_path:
+            try:
+                path = Path(self.csv_path)
+                path.parent.mkdir(parents=True, exist_ok=True)
+                self.fh = open(path, "w")
+                sel = ["-i", self.uuid] if self.uuid else []  # the UUID survives device remapping
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv", "-lms", "200", *sel],
+                    stdout=self.fh, stderr=subprocess.DEVNULL)
+            except (OSError, FileNotFoundError):
+                self.proc = None
         time.sleep(0.05)
         return self
 
@@ -322,7 +330,7 @@ def run_ours(args):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     stage_ms: dict = {}
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local, args.clocks_csv)
     with clocks:
         # headline: K steps, nothing between the library's kernels
         launches0 = blk.launch_count

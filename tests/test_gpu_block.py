@@ -104,12 +104,13 @@ def test_block_decode_after_prefill(cfg):
     blk.close()
 
 
+@pytest.mark.parametrize("lens0", [[5, 130, 257], [0, 1, 300]], ids=["ragged", "from-empty"])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_block_decode_ragged_lengths(dtype):
-    """Caller-filled caches of different lengths per sequence (set_lengths)."""
+def test_block_decode_ragged_lengths(dtype, lens0):
+    """Caller-filled caches of different lengths per sequence (set_lengths); a sequence
+    of length 0 decodes its first token, which attends to itself alone."""
     cfg = BlockConfig("ragged", d=256, n_heads=4, n_kv_heads=2, head_dim=64, f=512, B=3, T=1,
                       dtype=dtype, cache_len=300, gain="1+N(0,0.1)")
-    lens0 = [5, 130, 257]
     t_max = 320
     W = make_weights(cfg)
     k0, v0 = make_cache(cfg, t_max)

@@ -362,6 +362,24 @@ def test_decode_ragged_cache_lengths():
     np.testing.assert_allclose(dec["y"][:, 0], np.stack(want), rtol=1e-12, atol=1e-12)
 
 
+def test_decode_from_an_empty_cache_attends_to_itself():
+    """A first token decoded into an empty cache has one key: the softmax is 1 and each
+    query head's attention output is the new value vector of its KV head (GQA group)."""
+    H, Hkv, dh, d, f = 4, 2, 4, 8, 12
+    W = _tiny_weights(d, H, Hkv, dh, f, seed=72)
+    x = np.random.default_rng(73).normal(size=(2, 1, d))
+    kc = np.zeros((2, Hkv, 3, dh))
+    dec = ob.block_decode(x, W, H, Hkv, dh, 1e-6, 1e4, kc, kc.copy(), [0, 0])
+    rep = H // Hkv
+    for h in range(H):
+        np.testing.assert_allclose(dec["o"][:, 0, h * dh:(h + 1) * dh], dec["v_new"][:, h // rep, 0],
+                                   rtol=1e-12, atol=1e-12)
+    # and it is the one-token prefill
+    for b in range(2):
+        pre = ob.block_prefill(x[b:b + 1], W, H, Hkv, dh, 1e-6, 1e4)
+        np.testing.assert_allclose(dec["y"][b], pre["y"][0], rtol=1e-12, atol=1e-12)
+
+
 def test_kv_cache_bytes_ledger():
     """Chapter 04 memory accounting: L·2·B·T·H_kv·d_h·bytes equals the size of
     an allocated [layers,B,T,H_kv,D] K and V buffer pair (source-map layout)

@@ -91,6 +91,20 @@ lb_status llama_block_set_weights(llama_block* blk, const void* wq, const void* 
  * (LB_ERR_NO_WEIGHTS) and every K dimension a multiple of 64 (LB_ERR_UNSUPPORTED). */
 lb_status llama_block_quantize_decode_weights(llama_block* blk, int enable, void* stream);
 
+/* Dynamic NTK scaling of the rotary embedding (LMDrive page §2.2: the rotary module
+ * "supports dynamic NTK scaling" to extend the maximum sequence length; the pages give
+ * no formula). With original_max_pos = L0 > 0 and factor >= 1, a later prefill, extend
+ * or decode call whose longest sequence reaches L > L0 tokens rotates the Q and K of
+ * its new tokens with the base
+ *     base' = rope_base * (factor * L / L0 - (factor - 1)) ^ (head_dim / (head_dim - 2)),
+ * calls with L <= L0 with rope_base; keys already in the cache keep the rotation they
+ * were stored with. The handle rewrites the RoPE table rows a call reads (fp64 angles,
+ * one extra kernel on the call's stream). original_max_pos = 0 turns it off and
+ * restores the plain table on `stream`. LB_ERR_INVALID_ARG for a NULL handle,
+ * original_max_pos < 0, or factor < 1 (or not finite) when turning it on. */
+lb_status llama_block_set_rope_dynamic_ntk(llama_block* blk, float factor, int original_max_pos,
+                                           void* stream);
+
 /* Preallocate the workspace for up to `max_tokens` prefill rows (B*T) and
  * `max_batch` decode sequences, so that later calls allocate nothing (needed
  * before capturing calls in a CUDA graph). Optional: calls grow the workspace

@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "LB_F32", "LB_BF16", "LlamaBlockError", "lib", "lib_path", "dtype_code",
     "llama_block_create", "llama_block_set_weights", "llama_block_reserve",
-    "llama_block_quantize_decode_weights",
+    "llama_block_quantize_decode_weights", "llama_block_set_rope_dynamic_ntk",
     "llama_block_prefill", "llama_block_extend", "llama_block_decode", "llama_block_set_lengths",
     "llama_block_kv_cache_bytes", "llama_block_sync_status", "llama_block_destroy",
     "llama_block_last_error", "llama_block_selftest_timeout", "llama_block_enable_timing",
@@ -49,6 +49,7 @@ _SIGS = {
     "llama_block_set_weights": (_i, [_p] * 11),
     "llama_block_reserve": (_i, [_p, _i, _i]),
     "llama_block_quantize_decode_weights": (_i, [_p, _i, _p]),
+    "llama_block_set_rope_dynamic_ntk": (_i, [_p, _f, _i, _p]),
     "llama_block_tp_attn_prefill": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p]),
     "llama_block_tp_attn_decode": (_i, [_p, _p, _p, _i, _p, _p, _i, _p, _p]),
     "llama_block_tp_mlp": (_i, [_p, _p, _p, _p, _p, _i, _p]),
@@ -146,6 +147,12 @@ def llama_block_set_weights(h, wq, wk, wv, wo, w_gate, w_up, w_down, g_attn, g_m
 def llama_block_quantize_decode_weights(h, enable=True, stream=None):
     _check(lib.llama_block_quantize_decode_weights(h, 1 if enable else 0, _stream(stream)),
            "llama_block_quantize_decode_weights")
+
+
+def llama_block_set_rope_dynamic_ntk(h, factor, original_max_pos, stream=None):
+    """Dynamic NTK RoPE scaling (see the C header); original_max_pos = 0 turns it off."""
+    _check(lib.llama_block_set_rope_dynamic_ntk(h, float(factor), int(original_max_pos), _stream(stream)),
+           "llama_block_set_rope_dynamic_ntk")
 
 
 def llama_block_reserve(h, max_tokens, max_batch):
@@ -346,6 +353,9 @@ class LlamaBlock:
     def quantize_decode_weights(self, enable=True, stream=None):
         llama_block_quantize_decode_weights(self.handle, enable, stream)
 
+    def set_rope_dynamic_ntk(self, factor, original_max_pos, stream=None):
+        llama_block_set_rope_dynamic_ntk(self.handle, factor, original_max_pos, stream)
+
     def prefill(self, x, y, k_cache, v_cache, cache_len, stream=None):
         llama_block_prefill(self.handle, x, y, k_cache, v_cache, cache_len, stream)
 
@@ -457,6 +467,12 @@ class LlamaStack:
         """INT8 weight-only decode projections for every layer (or back to bf16)."""
         for layer in range(self.n_layers):
             llama_block_quantize_decode_weights(llama_stack_layer(self.handle, layer), enable, stream)
+
+    def set_rope_dynamic_ntk(self, factor, original_max_pos, stream=None):
+        """Dynamic NTK RoPE scaling for every layer (original_max_pos = 0: off)."""
+        for layer in range(self.n_layers):
+            llama_block_set_rope_dynamic_ntk(llama_stack_layer(self.handle, layer), factor,
+                                             original_max_pos, stream)
 
     def prefill(self, x, y, k_caches, v_caches, cache_len, stream=None):
         llama_stack_prefill(self.handle, x, y, k_caches, v_caches, cache_len, stream)

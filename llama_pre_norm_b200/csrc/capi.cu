@@ -160,6 +160,11 @@ struct llama_block {
   void *w_qkv = nullptr, *w_o = nullptr, *w_gu = nullptr, *w_d = nullptr;
   void *g1 = nullptr, *g2 = nullptr;
   float *cos_t = nullptr, *sin_t = nullptr;
+  // dynamic NTK RoPE scaling (llama_block_set_rope_dynamic_ntk): off when ntk_orig == 0;
+  // rope_mixed: some table rows hold another base than `base`
+  float ntk_factor = 1.f;
+  int ntk_orig = 0;
+  bool rope_mixed = false;
   int* err = nullptr;
   bool has_weights = false;
   void* ws = nullptr;
@@ -546,6 +551,28 @@ lb_status llama_block_quantize_decode_weights(llama_block* b, int enable, void* 
   return LB_OK;
 }
 
+lb_status llama_block_set_rope_dynamic_ntk(llama_block* b, float factor, int original_max_pos,
+                                           void* stream) {
+  if (!b) return fail(LB_ERR_INVALID_ARG, "set_rope_dynamic_ntk: NULL handle");
+  LB_ON_DEVICE(b, "set_rope_dynamic_ntk");
+  if (original_max_pos == 0) {  // off: plain RoPE everywhere again
+    b->ntk_orig = 0;
+    b->ntk_factor = 1.f;
+    if (b->rope_mixed) {
+      LB_CUDA(launch_rope_table(b->cos_t, b->sin_t, 0, b->max_pos, b->dh / 2, (double)b->base, b->dh,
+                                (cudaStream_t)stream));
+      b->rope_mixed = false;
+    }
+    return LB_OK;
+  }
+  if (original_max_pos < 0 || !(factor >= 1.f) || !std::isfinite(factor))
+    return fail(LB_ERR_INVALID_ARG,
+                "set_rope_dynamic_ntk: need factor >= 1 and original_max_pos > 0 (0 turns it off)");
+  b->ntk_factor = factor;
+  b->ntk_orig = original_max_pos;
+  return LB_OK;
+}
+
 lb_status llama_block_reserve(llama_block* b, int max_tokens, int max_batch) {
   if (!b) return fail(LB_ERR_INVALID_ARG, "reserve: NULL handle");
   LB_ON_DEVICE(b, "reserve");
@@ -560,6 +587,31 @@ lb_status llama_block_set_lengths(llama_block* b, const int32_t* lens_host, int 
   if (!b || !lens_host || B <= 0) return fail(LB_ERR_INVALID_ARG, "set_lengths: bad argument");
   b->lens.assign(lens_host, lens_host + B);
   return LB_OK;
+}
+
+// Dynamic NTK scaling (the rotary embedding of the LMDrive page §2.2 "supports dynamic
+// NTK scaling to extend the maximum sequence length"; the pages give no formula, the
+// reading taken is the dynamic NTK-aware rule): a call whose longest sequence reaches
+// L > L0 tokens (L0 = the trained context) rotates its new tokens with
+//   base' = base * (factor * L / L0 - (factor - 1)) ^ (dh / (dh - 2)),
+// which leaves the highest frequency alone and stretches the lowest one's wavelength by
+// exactly factor * L / L0 - (factor - 1); keys already in the cache keep their rotation.
+static double call_rope_base(const llama_block* b, int L) {
+  if (b->ntk_orig <= 0 || L <= b->ntk_orig) return (double)b->base;
+  const double s = (double)b->ntk_factor * L / b->ntk_orig - ((double)b->ntk_factor - 1.0);
+  return (double)b->base * std::pow(s, (double)b->dh / (double)(b->dh - 2));
+}
+
+// Whether a call reaching length L must first rewrite the table rows it reads.
+static bool rope_rows_stale(const llama_block* b, int L) {
+  return b->rope_mixed || call_rope_base(b, L) != (double)b->base;
+}
+
+// Rewrite table rows [p0, p1) for the base of a call reaching length L.
+static cudaError_t update_rope_rows(llama_block* b, int p0, int p1, int L, cudaStream_t s) {
+  const double base = call_rope_base(b, L);
+  if (base != (double)b->base) b->rope_mixed = true;
+  return launch_rope_table(b->cos_t, b->sin_t, p0, p1, b->dh / 2, base, b->dh, s);
 }
 
 static lb_status check_cache_args(llama_block* b, const void* x, const void* y, int B,
@@ -587,6 +639,8 @@ static lb_status run_prefill(llama_block* b, const void* x, void* y, int B, int 
   const int d = b->d, H = b->H, Hkv = b->Hkv, dh = b->dh, f = b->f;
 
   b->stage_names.clear();
+  if (rope_rows_stale(b, L + T))  // dynamic NTK: positions L .. L+T-1 for this call's base
+    LB_STAGE("rope_table", 1, update_rope_rows(b, L, L + T, L + T, s));
   if (b->dtype == kBF16) {
     // RMSNorm statistics of X (its gain is folded into W_qkv); also zeroes the X'
     // statistic accumulated by o_proj and sets cache_len = L + T.
@@ -691,6 +745,14 @@ lb_status llama_block_decode(llama_block* b, const void* x, void* y, int B, void
   const int d = b->d, H = b->H, Hkv = b->Hkv, dh = b->dh, f = b->f;
 
   b->stage_names.clear();
+  {  // dynamic NTK: the rows at the sequences' positions, for this step's base
+    int lo = b->lens[0], hi = b->lens[0] + 1;
+    for (int v : b->lens) {
+      lo = std::min(lo, v);
+      hi = std::max(hi, v + 1);
+    }
+    if (rope_rows_stale(b, hi)) LB_STAGE("rope_table", 1, update_rope_rows(b, lo, hi, hi, s));
+  }
   if (b->dtype == kBF16) {
     const DecodePlan plan = decode_plan(b, B, b->decode_int8);
     const int bn = plan.bn;
@@ -798,6 +860,7 @@ lb_status llama_block_tp_attn_prefill(llama_block* b, const void* x, void* o_par
   PrefillWs w = carve_prefill(b, b->ws, M, &need);
   const int d = b->d, H = b->H, Hkv = b->Hkv, dh = b->dh;
   b->stage_names.clear();
+  if (rope_rows_stale(b, T)) LB_STAGE("rope_table", 1, update_rope_rows(b, 0, T, T, s));
   LB_STAGE("row_stats_attn", 1, launch_row_ssq(x, w.ss1, w.ss2, M, d, cache_len, B, T, s));
   GemmEpi e1;
   e1.kind = kEpiQkvRope;
@@ -839,6 +902,14 @@ lb_status llama_block_tp_attn_decode(llama_block* b, const void* x, void* o_part
     return launch_gemm_tc(wbf, act, Mw, B, Kw, plan.bn, split, ep, b->num_sms, s);
   };
   b->stage_names.clear();
+  {  // dynamic NTK: the rows at the sequences' positions, for this step's base
+    int lo = b->lens[0], hi = b->lens[0] + 1;
+    for (int v : b->lens) {
+      lo = std::min(lo, v);
+      hi = std::max(hi, v + 1);
+    }
+    if (rope_rows_stale(b, hi)) LB_STAGE("rope_table", 1, update_rope_rows(b, lo, hi, hi, s));
+  }
   LB_STAGE("rmsnorm_attn", 1,
            launch_resid_rmsnorm(kBF16, x, nullptr, 0, 0, nullptr, nullptr, w.h, B, d, b->eps, s));
   GemmEpi e;

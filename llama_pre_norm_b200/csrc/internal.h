@@ -104,6 +104,9 @@ cudaError_t launch_resid_add(int dtype, const void* resid, const float* part, in
                              long long split_stride, void* out, long long total, int* lens, int B,
                              int len_inc, cudaStream_t s);
 cudaError_t launch_set_lens(int* lens, int B, int value, cudaStream_t s);
+// cos_t / sin_t rows [p0, p1) (each `half` = dh/2 wide) for rotary base `base`, in fp64.
+cudaError_t launch_rope_table(float* cos_t, float* sin_t, int p0, int p1, int half, double base,
+                              int dh, cudaStream_t s);
 // ss[m] = sum_j x[m][j]^2 (fp32) for bf16 rows; zeroes ss_zero[m] (when given) for a
 // later accumulation; block 0 also sets lens[0..B) = len_value (when lens given).
 cudaError_t launch_row_ssq(const void* x, float* ss, float* ss_zero, int rows, int d, int* lens,

@@ -6,7 +6,8 @@
 //     fp32 path,
 //   * SiLU(gate) * up from split-K partials (LlamaMLP, §2.4),
 //   * the final residual add (+ cache length increment for decode),
-//   * standalone RoPE (rotate_half pairing, §2.2).
+//   * standalone RoPE (rotate_half pairing, §2.2), and rows of the RoPE table for a
+//     given rotary base (dynamic NTK scaling).
 //
 // Every kernel reads 8-element vectors (one 16-byte access for bf16) and
 // accumulates in fp32; each stored value is rounded once.
@@ -360,6 +361,36 @@ __global__ void set_lens_kernel(int* lens, int B, int value) {
 
 cudaError_t launch_set_lens(int* lens, int B, int value, cudaStream_t s) {
   return launch_k(set_lens_kernel, (B + 127) / 128, 128, 0, s, lens, B, value);
+}
+
+// ---------------------------------------------------------------- RoPE table rows
+// Rows [p0, p1) of the RoPE table for rotary base `base` (LMDrive page §2.2
+// LlamaRotaryEmbedding: inv_freq_i = base^(-2i/dh), angle = pos * inv_freq_i): the angle
+// and its cosine and sine in fp64, stored as fp32 cos / sin [pos][dh/2], the same
+// construction as the table the handle builds at creation. Used by dynamic NTK scaling,
+// whose base depends on the length a call reaches.
+__global__ void rope_table_kernel(float* __restrict__ cos_t, float* __restrict__ sin_t, int p0,
+                                  int p1, int half, double base, int dh) {
+  pdl_wait();
+  pdl_trigger();
+  const long long n = (long long)(p1 - p0) * half;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int p = p0 + (int)(idx / half), i = (int)(idx % half);
+    const double inv = 1.0 / pow(base, (2.0 * i) / (double)dh);
+    double sv, cv;
+    sincos((double)p * inv, &sv, &cv);
+    cos_t[(long long)p * half + i] = (float)cv;
+    sin_t[(long long)p * half + i] = (float)sv;
+  }
+}
+
+cudaError_t launch_rope_table(float* cos_t, float* sin_t, int p0, int p1, int half, double base,
+                              int dh, cudaStream_t s) {
+  if (p1 <= p0 || half <= 0) return cudaSuccess;
+  const long long n = (long long)(p1 - p0) * half;
+  const int blocks = (int)std::min<long long>((n + 255) / 256, 148 * 8);
+  return launch_k(rope_table_kernel, blocks, 256, 0, s, cos_t, sin_t, p0, p1, half, base, dh);
 }
 
 // ---------------------------------------------------------------- RoPE (standalone)

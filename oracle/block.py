@@ -30,8 +30,10 @@ Readings where the pages are silent or disagree (each is listed in the design doc):
     length ([Mechanics] chapter 04, "position offset must follow the cache").
 
 Every function here is pinned by ``tests/test_oracle.py`` (worked examples from
-the pages, closed forms, invariants, and library routines on tiny inputs); no
-function is "parity unpinned".
+the pages, closed forms, invariants, and library routines on tiny inputs), except
+``dynamic_ntk_rope_base``: parity unpinned. [LMDrive] §2.2 names dynamic NTK
+scaling without a formula; that function is the reading taken, checked only
+against the invariants that define it.
 """
 
 from __future__ import annotations
@@ -69,6 +71,24 @@ def rmsnorm(x, g, eps: float) -> np.ndarray:
 def rope_inv_freq(head_dim: int, base: float) -> np.ndarray:
     exps = np.arange(0, head_dim, 2, dtype=np.float64) / head_dim
     return 1.0 / (float(base) ** exps)
+
+
+def dynamic_ntk_rope_base(base: float, head_dim: int, L: int, L0: int, factor: float) -> float:
+    """Rotary base for a call whose longest sequence reaches L tokens, under dynamic NTK
+    scaling with trained context L0 and scale factor `factor`.
+
+    PARITY UNPINNED: [LMDrive] §2.2 says the rotary module supports dynamic NTK scaling
+    to extend the maximum sequence length, and gives no formula. Reading taken (the
+    NTK-aware rule): up to L0 the base is unchanged; beyond it, with
+    s = factor * L / L0 - (factor - 1) (1 at L = L0), the base grows so that the
+    highest rotary frequency (base^0 = 1) stays put and the lowest one,
+    base^(-(d_h - 2) / d_h), slows down by exactly s. Solving
+    base'^(-(d_h - 2) / d_h) = base^(-(d_h - 2) / d_h) / s for base' gives the return value.
+    """
+    if L0 <= 0 or L <= L0:
+        return float(base)
+    s = factor * L / L0 - (factor - 1.0)
+    return float(base) * s ** (head_dim / (head_dim - 2.0))
 
 
 def rope_cos_sin(positions, head_dim: int, base: float):

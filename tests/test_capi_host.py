@@ -26,7 +26,7 @@ def declared_functions():
 
 def test_library_exports_every_declared_function():
     names = declared_functions()
-    assert "llama_block_create" in names and "causal_attn" in names and len(names) == 33
+    assert "llama_block_create" in names and "causal_attn" in names and len(names) == 34
     for n in names:
         assert hasattr(lb.lib, n), f"{n} declared in llama_block.h but not exported"
 
@@ -67,6 +67,7 @@ def test_create_null_out_and_null_handles():
     assert lb.lib.llama_block_decode(None, None, None, 1, None, None, 1, None, None) == 1
     assert lb.lib.llama_block_reserve(None, 1, 1) == 1
     assert lb.lib.llama_block_quantize_decode_weights(None, 1, None) == 1
+    assert lb.lib.llama_block_set_rope_dynamic_ntk(None, 2.0, 2048, None) == 1
     assert lb.lib.llama_block_tp_mlp(None, None, None, None, None, 1, None) == 1
     assert lb.lib.llama_block_tp_add(None, None, None, 4, 8, 1, None) == 1
     assert lb.lib.llama_block_tp_add(None, None, None, 4, 7, 1, None) == 1

@@ -380,6 +380,32 @@ def test_decode_from_an_empty_cache_attends_to_itself():
         np.testing.assert_allclose(dec["y"][b], pre["y"][0], rtol=1e-12, atol=1e-12)
 
 
+def test_dynamic_ntk_base_invariants():
+    """Dynamic NTK scaling (named, without a formula, by [LMDrive] §2.2; parity unpinned):
+    the invariants that define the reading taken. Up to the trained context the base is
+    unchanged and it is continuous there; beyond it the highest rotary frequency stays 1
+    and the lowest one slows down by exactly s = factor * L / L0 - (factor - 1); the base
+    grows with L and with the factor."""
+    base, L0 = 10000.0, 2048
+    for dh in (64, 128):
+        for factor in (1.0, 2.0, 4.0):
+            assert ob.dynamic_ntk_rope_base(base, dh, 1, L0, factor) == base
+            assert ob.dynamic_ntk_rope_base(base, dh, L0, L0, factor) == base
+            assert math.isclose(ob.dynamic_ntk_rope_base(base, dh, L0 + 1, L0, factor), base, rel_tol=5e-3)
+            prev = base
+            for L in (L0 + 1, 3000, 4096, 8192, 32768):
+                b2 = ob.dynamic_ntk_rope_base(base, dh, L, L0, factor)
+                s = factor * L / L0 - (factor - 1.0)
+                f0, f1 = ob.rope_inv_freq(dh, base), ob.rope_inv_freq(dh, b2)
+                assert f1[0] == 1.0
+                assert math.isclose(f1[-1], f0[-1] / s, rel_tol=1e-12)
+                assert np.all(np.diff(f1) < 0) and np.all(f1 <= f0)
+                assert b2 > prev
+                prev = b2
+        assert ob.dynamic_ntk_rope_base(base, dh, 4096, L0, 4.0) > ob.dynamic_ntk_rope_base(base, dh, 4096, L0, 2.0)
+    assert ob.dynamic_ntk_rope_base(base, 128, 4096, 0, 2.0) == base  # off
+
+
 def test_kv_cache_bytes_ledger():
     """Chapter 04 memory accounting: L·2·B·T·H_kv·d_h·bytes equals the size of
     an allocated [layers,B,T,H_kv,D] K and V buffer pair (source-map layout)

@@ -644,7 +644,7 @@ static lb_status run_prefill(llama_block* b, const void* x, void* y, int B, int 
   if (b->dtype == kBF16) {
     // RMSNorm statistics of X (its gain is folded into W_qkv); also zeroes the X'
     // statistic accumulated by o_proj and sets cache_len = L + T.
-    LB_STAGE("row_stats_attn", 1, launch_row_ssq(x, w.ss1, w.ss2, M, d, cache_len, B, L + T, s));
+    LB_STAGE("row_stats_attn", 1, launch_row_ssq(x, w.ss1, w.ss2, M, d, cache_len, B, L + T, b->err, s));
     GemmEpi e1;
     e1.kind = kEpiQkvRope;
     e1.T = T; e1.H = H; e1.Hkv = Hkv; e1.dh = dh; e1.t_max = t_max; e1.max_pos = b->max_pos;
@@ -861,7 +861,7 @@ lb_status llama_block_tp_attn_prefill(llama_block* b, const void* x, void* o_par
   const int d = b->d, H = b->H, Hkv = b->Hkv, dh = b->dh;
   b->stage_names.clear();
   if (rope_rows_stale(b, T)) LB_STAGE("rope_table", 1, update_rope_rows(b, 0, T, T, s));
-  LB_STAGE("row_stats_attn", 1, launch_row_ssq(x, w.ss1, w.ss2, M, d, cache_len, B, T, s));
+  LB_STAGE("row_stats_attn", 1, launch_row_ssq(x, w.ss1, w.ss2, M, d, cache_len, B, T, b->err, s));
   GemmEpi e1;
   e1.kind = kEpiQkvRope;
   e1.T = T; e1.H = H; e1.Hkv = Hkv; e1.dh = dh; e1.t_max = t_max; e1.max_pos = b->max_pos;

@@ -110,7 +110,7 @@ cudaError_t launch_rope_table(float* cos_t, float* sin_t, int p0, int p1, int ha
 // ss[m] = sum_j x[m][j]^2 (fp32) for bf16 rows; zeroes ss_zero[m] (when given) for a
 // later accumulation; block 0 also sets lens[0..B) = len_value (when lens given).
 cudaError_t launch_row_ssq(const void* x, float* ss, float* ss_zero, int rows, int d, int* lens,
-                           int B, int len_value, cudaStream_t s);
+                           int B, int len_value, int* err, cudaStream_t s);
 // w[r][c] = bf16(w[r][c] * g[c]) in place (bf16 [rows, cols], g [cols]).
 cudaError_t launch_scale_cols(void* w, const void* g, long long rows, int cols, cudaStream_t s);
 cudaError_t launch_rope_apply(int dtype, void* x, const int* pos, int B, int T, int H, int dh,

@@ -287,52 +287,70 @@ cudaError_t launch_add_rows(int dtype, const void* a, const void* b, void* out, 
 
 // ---------------------------------------------------------------- row statistics
 // Sum of squares of each bf16 row (the RMSNorm statistic; the GEMM that consumes
-// the row applies rsqrt(ss/d + eps) in its epilogue). One warp per row with all
-// of the row's 16-byte loads issued before the first use, so each SM keeps many
-// loads in flight.
-constexpr int kSsqWarps = 8;
-constexpr int kSsqMaxVec = 32;  // 16-byte vectors per lane: rows up to 32*8*32 = 8192
+// the row applies rsqrt(ss/d + eps) in its epilogue). A block takes kSsqRows rows:
+// one thread requests them whole from global memory with bulk asynchronous copies
+// into shared memory (one mbarrier, bytes counted on completion), then warp w sums
+// row w. The copy engine keeps far more bytes in flight per SM than per-thread
+// loads can, which is what a read-once kernel needs to reach HBM bandwidth.
+constexpr int kSsqRows = 4;
+constexpr int kSsqMaxD = 16384;  // widest row: 4 rows x 32 KB of shared memory
 
-__global__ void __launch_bounds__(kSsqWarps * 32) row_ssq_kernel(const bf16* __restrict__ x,
-                                                                 float* __restrict__ ss,
-                                                                 float* __restrict__ ss_zero,
-                                                                 int rows, int d, int* lens, int B,
-                                                                 int len_value) {
+__global__ void __launch_bounds__(kSsqRows * 32) row_ssq_kernel(const bf16* __restrict__ x,
+                                                                float* __restrict__ ss,
+                                                                float* __restrict__ ss_zero,
+                                                                int rows, int d, int* lens, int B,
+                                                                int len_value, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* buf = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const uint32_t row_bytes = (uint32_t)d * 2;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(buf + kSsqRows * row_bytes);
+  const long long row0 = (long long)blockIdx.x * kSsqRows;
+  const int nrows = rows - row0 < kSsqRows ? (int)(rows - row0) : kSsqRows;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
   pdl_wait();
   pdl_trigger();
   if (lens && blockIdx.x == 0)
     for (int b = threadIdx.x; b < B; b += blockDim.x) lens[b] = len_value;
-  const int lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * kSsqWarps + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const int nvec = d >> 3;
-  const uint4* src = reinterpret_cast<const uint4*>(x + row * d);
-  uint4 u[kSsqMaxVec];
-#pragma unroll
-  for (int i = 0; i < kSsqMaxVec; ++i)
-    if (lane + 32 * i < nvec) u[i] = src[lane + 32 * i];
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar, (uint32_t)nrows * row_bytes);
+    for (int r = 0; r < nrows; ++r)
+      bulk_load(buf + r * row_bytes, x + (row0 + r) * d, row_bytes, bar);
+  }
+  const bool ok = mbar_wait(bar, 0, err, 0x31);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (!ok || w >= nrows) return;
+  const uint4* src = reinterpret_cast<const uint4*>(buf + w * row_bytes);
   float acc = 0.f;
+  for (int i = lane; i < (d >> 3); i += 32) {
+    float v[8];
+    unpack_bf16x8(src[i], v);
 #pragma unroll
-  for (int i = 0; i < kSsqMaxVec; ++i) {
-    if (lane + 32 * i < nvec) {
-      float v[8];
-      unpack_bf16x8(u[i], v);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc = fmaf(v[e], v[e], acc);
-    }
+    for (int e = 0; e < 8; ++e) acc = fmaf(v[e], v[e], acc);
   }
   acc = warp_sum(acc);
   if (lane == 0) {
-    ss[row] = acc;
-    if (ss_zero) ss_zero[row] = 0.f;
+    ss[row0 + w] = acc;
+    if (ss_zero) ss_zero[row0 + w] = 0.f;
   }
 }
 
 cudaError_t launch_row_ssq(const void* x, float* ss, float* ss_zero, int rows, int d, int* lens,
-                           int B, int len_value, cudaStream_t s) {
+                           int B, int len_value, int* err, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  return launch_k(row_ssq_kernel, (rows + kSsqWarps - 1) / kSsqWarps, kSsqWarps * 32, 0, s,
-                  (const bf16*)x, ss, ss_zero, rows, d, lens, B, len_value);
+  if (d % 8 != 0 || d > kSsqMaxD || (reinterpret_cast<uintptr_t>(x) & 15) != 0)
+    return cudaErrorInvalidValue;
+  const int smem = kSsqRows * d * 2 + 16 + 128;
+  // the limit is raised once per device, so to what the widest supported row needs
+  static std::atomic<unsigned long long> attr_done{0};
+  if (cudaError_t e = ensure_smem_attr(row_ssq_kernel, kSsqRows * kSsqMaxD * 2 + 16 + 128, attr_done);
+      e != cudaSuccess)
+    return e;
+  return launch_k(row_ssq_kernel, (rows + kSsqRows - 1) / kSsqRows, kSsqRows * 32, smem, s,
+                  (const bf16*)x, ss, ss_zero, rows, d, lens, B, len_value, err);
 }
 
 // Fold an RMSNorm gain into the weights that consume the normalised row:

@@ -337,11 +337,6 @@ def block_extend(x, W: dict, n_heads: int, n_kv_heads: int, head_dim: int, eps: 
 
 
 # --------------------------------------------------------------------------
-# A stack of blocks — the "x L blocks" of the chapter-02 diagram of [Mechanics]
-# and the 32 decoder layers of [LMDrive] §1/§5: layer l's output is layer l+1's
-# input; each layer has its own KV cache.
-# --------------------------------------------------------------------------
-# --------------------------------------------------------------------------
 # Tensor parallelism — [Llama-MLP] §6.3: with Q/K/V and gate/up split by output rows
 # and o_proj and down by input columns, every rank's branch output is a partial sum;
 # an all-reduce over ranks completes the branch. A rank's slice is itself a block
@@ -369,6 +364,11 @@ def tp_mlp_partial(X1, Ws: dict, eps: float) -> np.ndarray:
     return swiglu_mlp(rmsnorm(X1, Ws["g_mlp"], eps), Ws["w_gate"], Ws["w_up"], Ws["w_down"])
 
 
+# --------------------------------------------------------------------------
+# A stack of blocks — the "x L blocks" of the chapter-02 diagram of [Mechanics]
+# and the 32 decoder layers of [LMDrive] §1/§5: layer l's output is layer l+1's
+# input; each layer has its own KV cache.
+# --------------------------------------------------------------------------
 def stack_prefill(X, Ws: list, n_heads: int, n_kv_heads: int, head_dim: int, eps: float,
                   rope_base: float) -> dict:
     """Prefill through len(Ws) layers. Returns y and the per-layer caches."""

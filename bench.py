@@ -330,7 +330,11 @@ def run_ours(args):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     stage_ms: dict = {}
-    clocks = ClockSampler(local, args.clocks_csv)
+    csv = args.clocks_csv
+    if csv and world > 1:  # one file per rank
+        path = Path(csv)
+        csv = str(path.with_name(f"{path.stem}_rank{rank}{path.suffix}"))
+    clocks = ClockSampler(local, csv)
     with clocks:
         # headline: K steps, nothing between the library's kernels
         launches0 = blk.launch_count

@@ -1,7 +1,7 @@
 """Tensor-parallel block ("深入解析Llama MLP模块" page §6.3) on one GPU: two shard handles
 (heads, KV heads and intermediate columns split in two, tp_shard_weights) stand for
 two ranks; the all-reduce of each branch's partial sums is the library's tp_add of
-the two partials (one GPU in this pool), and the block output y = x + o + m must match
+the two partials (both shards run on one GPU), and the block output y = x + o + m must match
 the fp64 oracle of the unsplit block, for a prefill and two decode steps, and every
 shard's cache must hold its KV heads. The decode steps also run with INT8 weights."""
 

@@ -20,7 +20,7 @@ Sources (page title, then section):
   [LlamaMLP] "深入解析Llama MLP模块：SwiGLU激活函数与参数配置详解": §3.3 (3df,
              no bias), §4.2 (gate gets SiLU, up does not, then down).
 
-Readings where the pages are silent or disagree (each is listed in the design doc):
+Readings where the pages are silent or disagree:
   * RoPE pairs dimension i with i + d_h/2 (rotate_half, [LMDrive] §2.2), not the
     interleaved (2i, 2i+1) pairs of [Mechanics] §02.2; the two differ by a fixed
     permutation of the head dimensions.

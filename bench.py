@@ -252,6 +252,14 @@ def cpu_oracle_sample(cfg, W=None, X=None) -> dict:
 
 
 # ------------------------------------------------------------------ reference arm
+def workload_config(cfg, world: int) -> dict:
+    """The `config` object of both arms' JSON lines: the 7B-shaped prefill workload."""
+    return {"workload": "llama7b block prefill, bf16, d=4096, 32 heads x 128, f=11008, B=1, T=2048",
+            "global_batch": cfg.B * world, "seq_len": cfg.T,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed before every timed step (256 MB write)"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -270,9 +278,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"llama7b block prefill, first {CPU_SAMPLE_T} of T=2048 tokens per step "
-                               "(fp64 CPU oracle)", "d": cfg.d, "n_heads": cfg.n_heads, "head_dim": cfg.head_dim,
-                   "f": cfg.f, "B": cfg.B, "T": CPU_SAMPLE_T},
+        "config": workload_config(cfg, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": samples[0]["cores"], "kind": "oracle",
                          "sample": samples[0]["sample"].rsplit(",", 1)[0]},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -506,10 +512,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,0.02) weights, N(0,1) input)",
-        "config": {"workload": "llama7b block prefill, bf16, d=4096, 32 heads x 128, f=11008, B=1, T=2048",
-                   "global_batch": cfg.B * world, "seq_len": cfg.T,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed before every timed step (256 MB write)"},
+        "config": workload_config(cfg, world),
         "prefill": {"tflops": flops["total"] / (ms_per_step * 1e-3) / 1e12,
                     "frac_of_bf16_peak": flops["total"] / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
                     "gflop_per_step": flops["total"] / 1e9, "stage_ms": stages},

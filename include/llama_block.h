@@ -198,6 +198,10 @@ lb_status llama_block_selftest_timeout(long long budget_ns, void* stream);
  * owns the caches. */
 typedef struct llama_stack llama_stack;
 
+/* Create a stack of n_layers blocks, each as llama_block_create(d, n_heads, n_kv_heads,
+ * head_dim, f, eps, rope_base, dtype, max_pos) on the current device; weights are set per
+ * layer through llama_stack_layer. Returns LB_ERR_INVALID_ARG for n_layers <= 0 or a null
+ * `out`, and any error of a layer's creation (the layers made so far are freed). */
 lb_status llama_stack_create(int n_layers, int d, int n_heads, int n_kv_heads, int head_dim,
                              int f, float eps, float rope_base, lb_dtype dtype, int max_pos,
                              llama_stack** out);

@@ -18,6 +18,13 @@ the copies on their own streams overlapping the neighbouring steps' compute.
 Multi-GPU runs are independent replicas (one process per GPU, no data-path
 collective): value = all ranks' tokens / the slowest rank's time.
 
+The other prefill shapes are timed the same way and reported beside the headline:
+``prefill_13b`` (d=5120, 40 heads, f=13824, B=4, T=1024), ``prefill_70b`` (d=8192,
+64 query / 8 KV heads, f=28672, B=1, T=4096) and ``prefill_tiny_f32`` (the fp32
+block, d=256, T=64), each with tokens/s, TFLOP/s, fraction of the bf16 peak, the
+per-stage times and, on a 1-GPU run, the fp64 oracle timed on 64 sampled rows per
+sequence with the GPU output's error at those rows.
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 ``--impl reference`` times the fp64 CPU oracle (the reference arm of this
@@ -44,12 +51,32 @@ L2_FLUSH_BYTES = 256 << 20
 CPU_SAMPLE_T = 2048  # tokens of the 7B prefill the CPU oracle evaluates per sample (the full T)
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the dominant
-# kernels, from one `ncu --set full` capture of the current kernels on this workload; set
-# to None whenever a kernel changes until it is captured again.
-NCU_TRAFFIC_BYTES = {
-    "gate_up_swiglu_gemm": 198_123_776 + 35_764_480,  # gemm_tc_pair_kernel<256, 2>, 7B prefill
-    "attention_decode": 2_148_352_000 + 8_126_464,    # attn_decode_split_kernel<128, 1>, L=4096
+# kernels, from one ncu capture on this workload (profiles/), with the SHA-256 prefix of
+# the kernel's source file at capture time: once that file changes the figure no longer
+# describes the kernel and the bench reports null until it is captured again.
+NCU_TRAFFIC = {
+    # gemm_tc_pair_kernel<256, 2>, 7B prefill
+    "gate_up_swiglu_gemm": {"bytes": 198_123_776 + 35_764_480, "source": "gemm_tc.cu",
+                            "sha256": None},
+    # attn_decode_split_kernel<128, 1>, L=4096
+    "attention_decode": {"bytes": 2_148_352_000 + 8_126_464, "source": "attn_decode.cu",
+                         "sha256": None},
 }
+
+
+def ncu_traffic(kernel: str):
+    """Captured DRAM bytes per launch of `kernel`, or None when its source changed since."""
+    import hashlib
+
+    t = NCU_TRAFFIC.get(kernel)
+    if not t:
+        return None
+    src = ROOT / "llama_pre_norm_b200" / "csrc" / t["source"]
+    try:
+        sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    except OSError:
+        return None
+    return t["bytes"] if sha == t["sha256"] else None
 
 
 def parse_args():
@@ -61,6 +88,8 @@ def parse_args():
     ap.add_argument("--decode-steps", type=int, default=128)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-configs", action="store_true",
+                    help="skip the 13B, 70B-GQA and fp32 tiny prefill lines")
     ap.add_argument("--clocks-csv", default=None,
                     help="also write nvidia-smi clock samples of the timed region to this CSV file")
     return ap.parse_args()
@@ -152,6 +181,7 @@ class ClockSampler:
         self._stop = None
         self._thread = None
         self.max_mhz = None
+        self._entered = False
 
     def _nvml_loop(self, handle, nv):
         import time as _t
@@ -185,13 +215,14 @@ class ClockSampler:
             try:
                 path = Path(self.csv_path)
                 path.parent.mkdir(parents=True, exist_ok=True)
-                self.fh = open(path, "w")
+                self.fh = open(path, "a" if self._entered else "w")
                 sel = ["-i", self.uuid] if self.uuid else []  # the UUID survives device remapping
                 self.proc = subprocess.Popen(
                     ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv", "-lms", "200", *sel],
                     stdout=self.fh, stderr=subprocess.DEVNULL)
             except (OSError, FileNotFoundError):
                 self.proc = None
+        self._entered = True
         time.sleep(0.05)
         return self
 
@@ -225,6 +256,50 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
+def host_info() -> dict:
+    """The host CPU the oracle runs on: logical cores, model name (lscpu), and the
+    BLAS threads numpy uses (the threads the oracle actually runs on)."""
+    model = None
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.strip().startswith("Model name:"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except (OSError, subprocess.SubprocessError):
+        pass
+    if model is None:
+        try:
+            with open("/proc/cpuinfo") as fh:
+                for line in fh:
+                    if line.startswith("model name"):
+                        model = line.split(":", 1)[1].strip()
+                        break
+        except OSError:
+            pass
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count() or 1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    return {"blas_threads": int(threads), "host_cores": os.cpu_count(), "cpu_model": model}
+
+
+def cpu_oracle_rows(cfg, W, X, rows) -> dict:
+    """Time the fp64 oracle on a row-sampled prefill: K and V projected for every
+    token (attention needs them), the query side, attention, o_proj and the MLP at
+    the sampled rows of every sequence. Returns the oracle output and the seconds."""
+    import numpy as np
+    import torch
+    from oracle import block as ob
+
+    Wn = {k: np.asarray(v.to(dtype=torch.float64).numpy()) for k, v in W.items()}
+    t0 = time.perf_counter()
+    ref = ob.block_prefill(X, Wn, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.eps, cfg.rope_base,
+                           rows=rows)
+    return {"ref": ref, "seconds": time.perf_counter() - t0}
+
+
 def cpu_oracle_sample(cfg, W=None, X=None) -> dict:
     """Time the fp64 oracle on the first CPU_SAMPLE_T tokens of the prefill
     workload (a complete causal prefill of that length). Returns tokens/s."""
@@ -232,11 +307,7 @@ def cpu_oracle_sample(cfg, W=None, X=None) -> dict:
     from oracle import block as ob
     from synth import make_weights, make_x
 
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count() or 1])
-    except Exception:
-        cores = os.cpu_count() or 1
+    host = host_info()
     if W is None:
         W = make_weights(cfg)
     if X is None:
@@ -246,7 +317,8 @@ def cpu_oracle_sample(cfg, W=None, X=None) -> dict:
     t0 = time.perf_counter()
     ob.block_prefill(Xs, Wn, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.eps, cfg.rope_base)
     dt = time.perf_counter() - t0
-    return {"value": cfg.B * CPU_SAMPLE_T / dt, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+    return {"value": cfg.B * CPU_SAMPLE_T / dt, "unit": UNIT, "cores": host["blas_threads"],
+            "host_cores": host["host_cores"], "cpu_model": host["cpu_model"], "kind": "oracle",
             "sample": f"fp64 numpy oracle, full prefill of the first {CPU_SAMPLE_T} tokens of the "
                       f"7B-shaped block (B=1), {dt:.2f} s", "seconds": dt}
 
@@ -258,6 +330,91 @@ def workload_config(cfg, world: int) -> dict:
             "global_batch": cfg.B * world, "seq_len": cfg.T,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": "flushed before every timed step (256 MB write)"}
+
+
+def bench_prefill_config(lb, cfg, args, peaks, dev, stream, flush, barrier, max_over_ranks,
+                         want_cpu: bool) -> dict:
+    """Time the prefill of one more workload shape like the headline (own handle, L2
+    flushed before every timed step, CUDA events on the library's stream, then a
+    second pass with the library's per-stage events) and, on rank 0 of a 1-GPU run,
+    the fp64 oracle on 64 sampled rows per sequence beside it (with the GPU output's
+    error at those rows)."""
+    import torch
+    from synth import make_weights, make_x, sample_rows
+
+    W = make_weights(cfg)
+    X = make_x(cfg)
+    dt = cfg.torch_dtype
+    blk = lb.LlamaBlock(cfg.d, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.f, cfg.eps, cfg.rope_base,
+                        dt, max_pos=cfg.T)
+    blk.set_weights({k: v.to(dev) for k, v in W.items()})
+    blk.reserve(cfg.B * cfg.T, cfg.B)
+    x = X.to(dev)
+    y = torch.empty_like(x)
+    kc = torch.zeros(cfg.B, cfg.n_kv_heads, cfg.T, cfg.head_dim, dtype=dt, device=dev)
+    vc = torch.zeros_like(kc)
+    lens = torch.zeros(cfg.B, dtype=torch.int32, device=dev)
+    for _ in range(args.warmup):
+        blk.prefill(x, y, kc, vc, lens)
+    blk.sync_status()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    l0 = blk.launch_count
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        blk.prefill(x, y, kc, vc, lens)
+        ends[i].record(stream)
+    barrier()
+    launches = blk.launch_count - l0
+    blk.sync_status()
+    ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends))) / args.steps
+    stage_ms: dict = {}
+    blk.enable_timing(True)
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        blk.prefill(x, y, kc, vc, lens)
+        for name, t in blk.stage_times():
+            stage_ms.setdefault(name, []).append(t)
+    barrier()
+    blk.enable_timing(False)
+    blk.sync_status()
+    flops = prefill_flops(cfg)
+    tflops = flops["total"] / (ms * 1e-3) / 1e12
+    stages = {k: round(statistics.mean(v), 4) for k, v in stage_ms.items()}
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    out = {"workload": f"{cfg.name}: {cfg.dtype}, d={cfg.d}, {cfg.n_heads} heads / {cfg.n_kv_heads} KV heads "
+                       f"x {cfg.head_dim}, f={cfg.f}, B={cfg.B}, T={cfg.T}",
+           "ms_per_step": ms, "tokens_per_s": replica_throughput(cfg.B * cfg.T, 1, world, ms),
+           "tflops": tflops, "gflop_per_step": flops["total"] / 1e9, "stage_ms": stages,
+           "steps": args.steps, "kernel_launches": launches}
+    if cfg.dtype == "bf16":
+        out["frac_of_bf16_peak"] = tflops / peaks["bf16_tflops"]
+        if "attention" in stages:
+            at = flops["attn"] / (stages["attention"] * 1e-3) / 1e12
+            out["attention"] = {"ms": stages["attention"], "gflop": flops["attn"] / 1e9, "tflops": at,
+                                "frac_of_bf16_peak": at / peaks["bf16_tflops"]}
+    if want_cpu:
+        import numpy as np
+
+        rows = sample_rows(cfg.T, 64, seed=11)
+        c = cpu_oracle_rows(cfg, W, X, rows)
+        got = y[:, rows].float().cpu().numpy()
+        want = c["ref"]["y"]
+        err = float(np.max(np.max(np.abs(got - want), axis=-1) / np.max(np.abs(want), axis=-1)))
+        host = host_info()
+        out["cpu_oracle"] = {"seconds": c["seconds"], "rows_per_sequence": len(rows),
+                             "sampled_rows_per_s": cfg.B * len(rows) / c["seconds"],
+                             "cores": host["blas_threads"], "host_cores": host["host_cores"],
+                             "cpu_model": host["cpu_model"], "kind": "oracle",
+                             "sample": ("fp64 numpy oracle, row-sampled: K/V projected for all "
+                                        f"{cfg.B * cfg.T} tokens, query side, attention, o_proj and "
+                                        f"MLP at {len(rows)} rows per sequence (first, last, seeded)")}
+        out["max_row_err_vs_oracle_at_sampled_rows"] = err
+    blk.close()
+    return out
 
 
 def run_reference(args):
@@ -280,6 +437,7 @@ def run_reference(args):
         "data": "synthetic",
         "config": workload_config(cfg, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": samples[0]["cores"], "kind": "oracle",
+                         "host_cores": samples[0]["host_cores"], "cpu_model": samples[0]["cpu_model"],
                          "sample": samples[0]["sample"].rsplit(",", 1)[0]},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -447,13 +605,12 @@ def run_ours(args):
                 "steps": args.decode_steps, "repetitions": reps, "kernel_launches": dec_launches,
                 "attention_kernel": {"ms": statistics.mean(attn_ms), "bytes_mean": attn_bytes_mean,
                                      "achieved_gbs": attn_gbs, "frac": attn_gbs / peaks["hbm_gbs"],
-                                     "traffic": NCU_TRAFFIC_BYTES["attention_decode"]},
+                                     "traffic": ncu_traffic("attention_decode")},
                 "int8_weights": {"ms_per_step": w8_step_ms, "hbm_gbs": w8_gbs,
                                  "frac_of_hbm": w8_gbs / peaks["hbm_gbs"], "bytes_per_step_mean": w8_bytes,
                                  "tokens_per_s": dcfg.B / (w8_step_ms * 1e-3) * world,
                                  "speedup_vs_bf16": per_step_ms / w8_step_ms, "kernel_launches": w8_launches},
             }
-    clk = clocks.summary()
 
     # ---------------- e2e: host buffers in and out through the public API, every step's
     # H2D copy of its input and D2H copy of its output inside the timed region. As a
@@ -494,6 +651,22 @@ def run_ours(args):
     barrier()
     e2e_tot = max_over_ranks(t_start.elapsed_time(t_end))
     blk.sync_status()
+    blk.close()
+    del xd, yd, kc, vc
+
+    # ---------------- the other prefill shapes (13B batched, 70B GQA, fp32 tiny), each timed
+    # like the headline, with the row-sampled CPU oracle beside it
+    extra = {}
+    if not args.no_extra_configs:
+        from synth import LLAMA13B, LLAMA70B, TINY_F32
+
+        want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+        with clocks:
+            for key, c in (("prefill_13b", LLAMA13B), ("prefill_70b", LLAMA70B), ("prefill_tiny_f32", TINY_F32)):
+                extra[key] = bench_prefill_config(lb, c, args, peaks, dev, stream, flush, barrier,
+                                                  max_over_ranks, want_cpu)
+                torch.cuda.empty_cache()
+    clk = clocks.summary()
 
     tokens = cfg.B * cfg.T
     flops = prefill_flops(cfg)
@@ -506,7 +679,7 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         c = cpu_oracle_sample(cfg, W, X)
-        cpu = {k: c[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        cpu = {k: c[k] for k in ("value", "unit", "cores", "host_cores", "cpu_model", "kind", "sample")}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -517,22 +690,25 @@ def run_ours(args):
                     "frac_of_bf16_peak": flops["total"] / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
                     "gflop_per_step": flops["total"] / 1e9, "stage_ms": stages},
         "decode": dec,
+        **extra,
         "roofline": {"kernel": "gate_up_swiglu_gemm", "bound": "tensor", "achieved": gu_tflops,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": gu_tflops / peaks["bf16_tflops"],
-                     "traffic": NCU_TRAFFIC_BYTES["gate_up_swiglu_gemm"],
+                     "traffic": ncu_traffic("gate_up_swiglu_gemm"),
                      "peak_source": f"{peaks['source']} bf16 burst (kernel timed alone within a short step)",
                      "algorithmic_flop_per_launch": flops["gate_up"]},
         "cpu_baseline": cpu,
         "e2e": {"value": replica_throughput(tokens, args.steps, world, e2e_tot), "unit": UNIT,
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": X.numel() * 2,
                 "ms_per_step": e2e_tot / args.steps,
-                "overlap": "H2D of step i+1 and D2H of step i-1 run on their own streams during step i"},
+                "overlap": "H2D of step i+1 and D2H of step i-1 run on their own streams during step i",
+                "path": "pinned host buffers copied by torch (cudaMemcpyAsync on side streams) around the "
+                        "device-pointer C-ABI call llama_block_prefill"},
         "gpu_launches": prefill_launches + (dec["kernel_launches"] + dec["int8_weights"]["kernel_launches"]
-                                            if dec else 0),
-        "gpu_launches_note": "library kernels launched in the timed prefill steps and the timed decode repetitions",
+                                            if dec else 0) + sum(e["kernel_launches"] for e in extra.values()),
+        "gpu_launches_note": ("library kernels launched in the timed prefill steps, the timed decode "
+                              "repetitions and the timed steps of the other prefill shapes"),
         "clocks": clk,
     }
-    blk.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -26,8 +26,9 @@
  *    reason is available from llama_block_last_error() (thread-local string).
  *  - Device-side waits are bounded: a wait that runs out latches an error word on
  *    the device instead of hanging; llama_block_sync_status() reads it.
- *  - Restrictions: head_dim in {64, 128}; n_heads / n_kv_heads in {1, 2, 4, 8};
- *    n_heads * head_dim and d are multiples of 64 for LB_BF16; y must not alias x.
+ *  - Restrictions: head_dim in {64, 128}; n_kv_heads divides n_heads (any
+ *    quotient); n_heads * head_dim and d are multiples of 64 for LB_BF16; y must
+ *    not alias x.
  *  - A handle is not thread-safe: do not call it concurrently from several threads.
  */
 #ifndef LLAMA_BLOCK_H
@@ -64,8 +65,8 @@ typedef struct llama_block llama_block; /* opaque, library-owned */
  * and leaves the caller's current device as it was. Its buffers and stream arguments
  * must belong to that device.
  * Returns LB_ERR_INVALID_ARG for non-positive sizes or a null `out`,
- * LB_ERR_UNSUPPORTED for head_dim not in {64,128} or n_heads / n_kv_heads not in
- * {1, 2, 4, 8}. */
+ * LB_ERR_UNSUPPORTED for head_dim not in {64,128} or n_heads not a multiple of
+ * n_kv_heads. */
 lb_status llama_block_create(int d, int n_heads, int n_kv_heads, int head_dim, int f,
                              float eps, float rope_base, lb_dtype dtype, int max_pos,
                              llama_block** out);
@@ -153,8 +154,10 @@ lb_status llama_block_set_lengths(llama_block* blk, const int32_t* lens_host, in
 size_t llama_block_kv_cache_bytes(int B, int n_kv_heads, int head_dim, int t_max,
                                   lb_dtype dtype);
 
-/* Synchronise `stream`, read and clear the device error word (of the handle, or
- * of the standalone entry points when blk is NULL). Returns LB_OK, LB_ERR_TIMEOUT
+/* Synchronise `stream`, read and clear the device error word (of the handle, or,
+ * when blk is NULL, the words of the current device's standalone entry points:
+ * the one they share and the one of decode_attn_static_scratch; with blk NULL
+ * this call allocates nothing). Returns LB_OK, LB_ERR_TIMEOUT
  * (a bounded wait ran out), LB_ERR_CACHE_FULL (a device-side bounds guard fired:
  * a cache index or RoPE position out of range; the write was skipped) or
  * LB_ERR_CUDA; details in last_error. */
@@ -312,20 +315,24 @@ lb_status swiglu_mlp(const void* h, const void* w_gate, const void* w_up,
  *
  * Computes, for each sequence b and query head h, the attention of the single
  * query q[b][h] (at position kv_len[b]) over keys 0..kv_len[b]:
- *   q: [B, n_heads, head_dim]; k, v: [B, n_kv_heads, k_stride_T, head_dim];
- *   kv_len: device int32 [B], kv_len[b] + 1 <= k_stride_T;
+ *   q: [B, n_heads, head_dim]; k, v: [B, n_kv_heads, k_stride_T, head_dim],
+ *   16-byte aligned; kv_len: device int32 [B], 0 <= kv_len[b] < k_stride_T;
  *   o: [B, n_heads * head_dim]; all bf16 except kv_len. The caller passes inputs
  *   and outputs; the split-KV partials go to a fixed array inside the library.
  * Limit: B * n_heads * ceil(k_stride_T / 512) * (head_dim + 2) <= 6 * 2^20 floats
- * (24 MiB); larger calls return LB_ERR_INVALID_ARG before anything is launched.
+ * (24 MiB); larger calls return LB_ERR_INVALID_ARG before anything is launched,
+ * as do misaligned k or v.
  * Every GPU that loads the library holds that array until the process exits.
  * The first call on a device looks up the array's device address on that
- * device; make that first call before any stream capture. All calls on one
- * device share its array and it keeps the last call's contents, so calls that
- * may overlap on that GPU (several streams, threads or processes) race:
- * serialise them.
- * A bounded wait that runs out ends the kernel early and sets a device word
- * private to this entry point; the output of that call is then undefined. */
+ * device; make that first call before any stream capture. The array belongs to
+ * the process's context on that device, so all calls of one process on one
+ * device share it and it keeps the last call's contents: calls that may overlap
+ * on that GPU (several streams, or several host threads) race, so serialise
+ * them. Separate processes each have their own copy.
+ * Errors found on the device (a kv_len[b] outside [0, k_stride_T), or a bounded
+ * wait that ran out) set a device word private to this entry point and leave
+ * that call's output undefined; llama_block_sync_status(NULL, stream) reads and
+ * clears it (LB_ERR_CACHE_FULL or LB_ERR_TIMEOUT), allocating nothing. */
 lb_status decode_attn_static_scratch(const void* q, const void* k, const void* v, void* o,
                                      const int32_t* kv_len, int B, int n_heads, int n_kv_heads,
                                      int head_dim, int k_stride_T, void* stream);

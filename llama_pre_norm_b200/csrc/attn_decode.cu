@@ -4,13 +4,16 @@
 //
 // The step is bound by the HBM read of K and V (each sequence reads
 // 2 * (L+1) * H_kv * d_h * 2 bytes), so the kernel is shaped to keep HBM busy:
-//   * split-KV: one CTA per (512-key split, KV head, sequence);
+//   * split-KV: one CTA per (512-key split, group of G query heads, sequence);
 //   * a producer warp streams the split through a 3-stage shared-memory ring of
 //     64-key chunks (K and V rows are contiguous in the [B, H_kv, t_max, d_h]
 //     cache, so each chunk is two bulk async copies), while
 //   * eight consumer warps each own 8 keys of every chunk and keep their own
-//     online-softmax state (running max, sum and output) for the n_rep query heads
-//     of the KV head, so no block-wide reduction sits inside the key loop:
+//     online-softmax state (running max, sum and output) for G query heads of the
+//     KV head, so no block-wide reduction sits inside the key loop. G is the
+//     largest of 8, 4, 2, 1 that divides n_rep = H / H_kv, so one CTA serves the
+//     whole group when n_rep is 1, 2, 4 or 8 and n_rep / G CTAs share it otherwise
+//     (any n_rep works; for n_rep = 3, 5, ... each CTA serves one query head):
 //       scores: lane = (key, quarter of d_h); 16-byte K reads rotated per lane so a
 //               quarter-warp hits 8 different banks; q held pre-rotated in registers;
 //       P V:    lane = d_h/32 consecutive dims; a warp reads whole V rows;
@@ -28,9 +31,12 @@ constexpr int kDecStages = 3;
 constexpr int kDecSplitKeys = 512;    // keys per CTA
 constexpr int kDecWarps = 8;          // consumer warps (8 keys of each chunk apiece)
 constexpr int kDecThreads = (kDecWarps + 1) * 32;
-constexpr int kMaxRep = 8;
 
 int decode_attn_chunks(int k_stride) { return (k_stride + kDecSplitKeys - 1) / kDecSplitKeys; }
+
+int decode_attn_heads_per_cta(int n_rep) {
+  return n_rep % 8 == 0 ? 8 : n_rep % 4 == 0 ? 4 : n_rep % 2 == 0 ? 2 : 1;
+}
 
 template <int DH>
 constexpr int dec_smem_bytes(int nrep) {
@@ -42,6 +48,8 @@ __global__ void __launch_bounds__(kDecThreads, NREP >= 4 ? 1 : 2) attn_decode_sp
     const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
     float* __restrict__ part, int H, int Hkv, int k_stride, int n_splits,
     const int* __restrict__ kv_len, float scale_log2, int* err) {
+  // NREP: query heads of this CTA (G above); they are heads hq0 .. hq0 + NREP - 1,
+  // all in the group of KV head hk.
   constexpr int QD = DH / 4;           // dims per lane in the score phase
   constexpr int QC = QD / 8;           // 16-byte chunks per lane (4 or 2)
   constexpr int VD = DH / 32;          // dims per lane in the P V phase (4 or 2)
@@ -54,15 +62,19 @@ __global__ void __launch_bounds__(kDecThreads, NREP >= 4 ? 1 : 2) attn_decode_sp
 
   pdl_wait();
   pdl_trigger();
-  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int split = blockIdx.x, b = blockIdx.z;
+  const int hq0 = blockIdx.y * NREP;
+  const int hk = hq0 / (H / Hkv);
   const int nkeys = kv_len[b] + 1;  // cached keys plus the one just appended
   const int k0 = split * kDecSplitKeys;
   const int nk = min(kDecSplitKeys, nkeys - k0);
   const long long head_stride = (long long)n_splits * (DH + 2);
-  float* out_base = part + (((long long)b * H + hk * NREP) * n_splits + split) * (DH + 2);
+  float* out_base = part + (((long long)b * H + hq0) * n_splits + split) * (DH + 2);
 
   if (nk <= 0 || nkeys > k_stride) {
-    if (nkeys > k_stride && threadIdx.x == 0 && split == 0) latch_error(err, kErrCacheBounds);
+    // a length outside [0, k_stride) is an error; the split then reads nothing
+    if ((nkeys > k_stride || nkeys <= 0) && threadIdx.x == 0 && split == 0)
+      latch_error(err, kErrCacheBounds);
     if (threadIdx.x < NREP) {  // empty split: contributes nothing to the combine
       out_base[threadIdx.x * head_stride + DH] = -INFINITY;
       out_base[threadIdx.x * head_stride + DH + 1] = 0.f;
@@ -80,7 +92,7 @@ __global__ void __launch_bounds__(kDecThreads, NREP >= 4 ? 1 : 2) attn_decode_sp
     fence_mbar_init();
   }
   for (int e = threadIdx.x; e < NREP * DH; e += kDecThreads)
-    qs[e] = __bfloat162float(q[((long long)b * H + hk * NREP) * DH + e]) * scale_log2;
+    qs[e] = __bfloat162float(q[((long long)b * H + hq0) * DH + e]) * scale_log2;
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -261,6 +273,10 @@ __global__ void attn_decode_combine_kernel(const float* __restrict__ part, bf16*
   pdl_trigger();
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const int used = min(n_splits, (kv_len[b] + 1 + kDecSplitKeys - 1) / kDecSplitKeys);
+  if (used <= 0) {  // negative length: the split kernel latched an error; write zeros
+    o[((long long)b * H + h) * DH + d] = __float2bfloat16_rn(0.f);
+    return;
+  }
   const float* base = part + ((long long)b * H + h) * n_splits * (DH + 2);
   float M = -INFINITY;
   for (int c = 0; c < used; ++c) M = fmaxf(M, base[c * (DH + 2) + DH]);
@@ -293,14 +309,14 @@ static cudaError_t run_decode(const void* q, const void* k, const void* v, void*
                               cudaStream_t s) {
   const int n_splits = decode_attn_chunks(k_stride);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
-  const dim3 grid(n_splits, Hkv, B);
+  const int g = decode_attn_heads_per_cta(H / Hkv);
+  const dim3 grid(n_splits, H / g, B);
   cudaError_t e;
-  switch (H / Hkv) {
+  switch (g) {
     case 1: e = run_split<DH, 1>(grid, q, k, v, part, H, Hkv, k_stride, n_splits, kv_len, scale_log2, err, s); break;
     case 2: e = run_split<DH, 2>(grid, q, k, v, part, H, Hkv, k_stride, n_splits, kv_len, scale_log2, err, s); break;
     case 4: e = run_split<DH, 4>(grid, q, k, v, part, H, Hkv, k_stride, n_splits, kv_len, scale_log2, err, s); break;
-    case 8: e = run_split<DH, 8>(grid, q, k, v, part, H, Hkv, k_stride, n_splits, kv_len, scale_log2, err, s); break;
-    default: return cudaErrorInvalidValue;
+    default: e = run_split<DH, 8>(grid, q, k, v, part, H, Hkv, k_stride, n_splits, kv_len, scale_log2, err, s); break;
   }
   if (e != cudaSuccess) return e;
   return launch_k(attn_decode_combine_kernel<DH>, dim3(H, B), DH, 0, s, (const float*)part,
@@ -311,8 +327,7 @@ cudaError_t launch_attn_decode(const void* q, const void* k, const void* v, void
                                int B, int H, int Hkv, int dh, int k_stride, const int* kv_len,
                                int* err, cudaStream_t s) {
   if (B <= 0) return cudaSuccess;
-  const int rep = H / Hkv;
-  if (rep != 1 && rep != 2 && rep != 4 && rep != 8) return cudaErrorInvalidValue;
+  if (Hkv <= 0 || H % Hkv) return cudaErrorInvalidValue;
   if (dh == 128) return run_decode<128>(q, k, v, o, part, B, H, Hkv, k_stride, kv_len, err, s);
   if (dh == 64) return run_decode<64>(q, k, v, o, part, B, H, Hkv, k_stride, kv_len, err, s);
   return cudaErrorInvalidValue;

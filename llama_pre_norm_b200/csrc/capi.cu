@@ -136,6 +136,15 @@ struct DeviceGuard {
 static std::mutex g_err_mu;
 static std::map<int, int*> g_err_words;
 
+// The standalone word of the current device if a call has created it (allocates nothing).
+static int* existing_standalone_err_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  auto it = g_err_words.find(dev);
+  return it == g_err_words.end() ? nullptr : it->second;
+}
+
 static int* standalone_err_word() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
@@ -358,11 +367,6 @@ lb_status llama_block_create(int d, int n_heads, int n_kv_heads, int head_dim, i
     return fail(LB_ERR_UNSUPPORTED, "create: head_dim %d not in {64,128}", head_dim);
   if (n_heads % n_kv_heads != 0)
     return fail(LB_ERR_UNSUPPORTED, "create: n_heads %% n_kv_heads != 0");
-  {
-    const int rep = n_heads / n_kv_heads;
-    if (rep != 1 && rep != 2 && rep != 4 && rep != 8)
-      return fail(LB_ERR_UNSUPPORTED, "create: query heads per KV head must be 1, 2, 4 or 8");
-  }
   if (d % 8 != 0 || d > 8192)
     return fail(LB_ERR_UNSUPPORTED, "create: d must be a multiple of 8 and <= 8192");
   if (dtype == LB_BF16 && (d % 64 != 0 || f % 8 != 0 || (n_heads * head_dim) % 64 != 0))
@@ -1030,17 +1034,35 @@ static const char* describe_err(int code) {
   return "a device-side bounds guard fired (cache index or RoPE position out of range)";
 }
 
+// Read a device error word and clear it when it is set.
+static cudaError_t take_err_word(int* word, int* code) {
+  *code = 0;
+  if (!word) return cudaSuccess;
+  cudaError_t e = cudaMemcpy(code, word, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && *code != 0) e = cudaMemset(word, 0, sizeof(int));
+  return e;
+}
+
+static cudaError_t noalloc_take_error(int* code);  // decode_attn_static_scratch's word
+
 lb_status llama_block_sync_status(llama_block* b, void* stream) {
   DeviceGuard dg(b ? b->device : -1);
   if (b && !dg.ok) return fail(LB_ERR_CUDA, "sync_status: cannot select the handle's device");
-  int* word = b ? b->err : standalone_err_word();
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return fail(LB_ERR_CUDA, "sync_status: %s", cudaGetErrorString(e));
-  if (!word) return fail(LB_ERR_CUDA, "sync_status: no error word");
   int code = 0;
-  LB_CUDA(cudaMemcpy(&code, word, sizeof(int), cudaMemcpyDeviceToHost));
+  if (b) {
+    LB_CUDA(take_err_word(b->err, &code));
+  } else {
+    // the standalone entry points of the current device: the word they share (looked up,
+    // never created here, so this allocates nothing) and the allocation-free decode
+    // attention's own word; both are cleared, the first code set is reported
+    int c_noalloc = 0;
+    LB_CUDA(take_err_word(existing_standalone_err_word(), &code));
+    LB_CUDA(noalloc_take_error(&c_noalloc));
+    if (code == 0) code = c_noalloc;
+  }
   if (code == 0) return LB_OK;
-  LB_CUDA(cudaMemset(word, 0, sizeof(int)));
   const bool wait = code >= kErrWaitBase && code < kErrWaitBase + 0x100;
   return fail(wait ? LB_ERR_TIMEOUT : LB_ERR_CACHE_FULL, "device error 0x%x: %s", code,
               describe_err(code));
@@ -1094,6 +1116,8 @@ lb_status causal_attn(const void* q, const void* k, const void* v, void* o, int 
   if (head_dim != 64 && head_dim != 128)
     return fail(LB_ERR_UNSUPPORTED, "causal_attn: head_dim %d not in {64,128}", head_dim);
   if (n_heads % n_kv_heads) return fail(LB_ERR_UNSUPPORTED, "causal_attn: n_heads %% n_kv_heads");
+  if (dtype == LB_BF16 && (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o) & 15))
+    return fail(LB_ERR_INVALID_ARG, "causal_attn: bf16 q, k, v and o must be 16-byte aligned");
   cudaStream_t s = (cudaStream_t)stream;
   if (dtype == LB_BF16) {
     int* err = standalone_err_word();
@@ -1339,6 +1363,21 @@ struct NoAllocSlot {
 static std::mutex g_noalloc_mu;
 static std::map<int, NoAllocSlot> g_noalloc_slots;
 
+// Read and clear the current device's word (nothing to read before the first call there).
+static cudaError_t noalloc_take_error(int* code) {
+  *code = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int* word = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    auto it = g_noalloc_slots.find(dev);
+    if (it != g_noalloc_slots.end()) word = it->second.err;
+  }
+  return take_err_word(word, code);
+}
+
 extern "C" lb_status decode_attn_static_scratch(const void* q, const void* k, const void* v,
                                                 void* o, const int32_t* kv_len, int B,
                                                 int n_heads, int n_kv_heads, int head_dim,
@@ -1349,11 +1388,10 @@ extern "C" lb_status decode_attn_static_scratch(const void* q, const void* k, co
     return fail(LB_ERR_INVALID_ARG, "decode_attn_static_scratch: sizes must be positive");
   if (head_dim != 64 && head_dim != 128)
     return fail(LB_ERR_UNSUPPORTED, "decode_attn_static_scratch: head_dim %d not in {64,128}", head_dim);
-  if (n_heads % n_kv_heads ||
-      (n_heads / n_kv_heads != 1 && n_heads / n_kv_heads != 2 && n_heads / n_kv_heads != 4 &&
-       n_heads / n_kv_heads != 8))
-    return fail(LB_ERR_UNSUPPORTED, "decode_attn_static_scratch: query heads per KV head must be "
-                                    "1, 2, 4 or 8");
+  if (n_heads % n_kv_heads)
+    return fail(LB_ERR_UNSUPPORTED, "decode_attn_static_scratch: n_heads %% n_kv_heads != 0");
+  if (((uintptr_t)k | (uintptr_t)v) & 15)
+    return fail(LB_ERR_INVALID_ARG, "decode_attn_static_scratch: k and v must be 16-byte aligned");
   const size_t need = (size_t)B * n_heads * decode_attn_chunks(k_stride_T) * (head_dim + 2);
   if (need > kNoAllocScratchFloats)
     return fail(LB_ERR_INVALID_ARG,

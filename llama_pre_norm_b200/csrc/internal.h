@@ -209,6 +209,8 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* o,
 // 0..kv_len[b] (the new key already appended). q [B,H,dh]; k,v [B,Hkv,k_stride,dh];
 // o [B, H*dh]. `part` holds B*H*max_chunks*(dh+2) floats.
 int decode_attn_chunks(int k_stride);
+// Query heads one decode-attention CTA serves: the largest of 8, 4, 2, 1 dividing n_rep.
+int decode_attn_heads_per_cta(int n_rep);
 cudaError_t launch_attn_decode(const void* q, const void* k, const void* v, void* o, float* part,
                                int B, int H, int Hkv, int dh, int k_stride, const int* kv_len,
                                int* err, cudaStream_t s);

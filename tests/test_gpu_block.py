@@ -30,6 +30,20 @@ SMALL_BF16 = [
                 dtype="bf16", gain="1+N(0,0.1)"),
 ]
 
+# GQA groupings outside {1, 2, 4, 8} (repeat_kv allows any n_rep = H / H_kv): the decode
+# attention then serves one (n_rep = 3) or two (n_rep = 6) query heads per CTA, or all
+# 16 with eight per CTA
+GQA_ANY = [
+    BlockConfig("bf16-rep3", d=512, n_heads=6, n_kv_heads=2, head_dim=64, f=1024, B=2, T=150,
+                dtype="bf16", gain="1+N(0,0.1)"),
+    BlockConfig("bf16-rep6", d=768, n_heads=12, n_kv_heads=2, head_dim=64, f=1024, B=1, T=300,
+                dtype="bf16"),
+    BlockConfig("bf16-rep16", d=1024, n_heads=16, n_kv_heads=1, head_dim=64, f=1536, B=1, T=200,
+                dtype="bf16"),
+    BlockConfig("f32-rep3", d=384, n_heads=6, n_kv_heads=2, head_dim=64, f=512, B=1, T=70,
+                dtype="f32", gain="1+N(0,0.1)"),
+]
+
 
 def _oracle_prefill(cfg, X, W):
     return ob.block_prefill(X, W, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.eps, cfg.rope_base)
@@ -57,7 +71,7 @@ def _check(cfg, got, want):
     assert row_err(got, want) <= _tol(cfg)
 
 
-@pytest.mark.parametrize("cfg", [TINY_F32] + SMALL_BF16, ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", [TINY_F32] + SMALL_BF16 + GQA_ANY, ids=lambda c: c.name)
 def test_block_prefill(cfg):
     W = make_weights(cfg)
     X = make_x(cfg)
@@ -73,7 +87,8 @@ def test_block_prefill(cfg):
     blk.close()
 
 
-@pytest.mark.parametrize("cfg", [TINY_F32.with_(B=2, T=40)] + SMALL_BF16[:2], ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", [TINY_F32.with_(B=2, T=40)] + SMALL_BF16[:2] + GQA_ANY,
+                         ids=lambda c: c.name)
 def test_block_decode_after_prefill(cfg):
     """Prefill T tokens, then decode 3 tokens; each decode output equals the
     oracle's decode (and hence the last row of a full recompute)."""

@@ -10,8 +10,9 @@ projections.
 One step = one prefill of the whole block (RMSNorm, fused QKV GEMM with RoPE and
 the KV-cache scatter, causal attention, o_proj + residual, RMSNorm, gate/up GEMM
 with SiLU*up, down_proj + residual) over the synthetic 2048-token input, called
-through the C ABI. Inputs are resident in HBM; L2 is flushed (256 MB write)
-before every timed step; each step is timed with CUDA events on the library's
+through the C ABI. Inputs are resident in HBM; L2 is flushed (a 256 MB write,
+then a 256 MB read, so that no dirty lines are left to write back) before every
+timed step; each step is timed with CUDA events on the library's
 stream. The ``e2e`` figure runs the same steps from pinned host buffers through the
 public API, each step's H2D input copy and D2H output copy inside the timed region,
 the copies on their own streams overlapping the neighbouring steps' compute.
@@ -140,6 +141,24 @@ def decode_bytes(cfg, L: int, int8_weights: bool = False) -> int:
 
 def decode_attn_bytes(cfg, L: int) -> int:
     return 2 * cfg.B * cfg.n_kv_heads * (L + 1) * cfg.head_dim * 2
+
+
+# ------------------------------------------------------------------ L2 flush
+class L2Flush:
+    """Evicts L2 outside the timed interval: a write of one buffer larger than L2,
+    then a read of another, so that the lines left in L2 when the timed step starts
+    are clean lines of unrelated data (the write alone would leave dirty lines whose
+    write-back the step's first kernel would pay for)."""
+
+    def __init__(self, nbytes: int, device):
+        import torch
+
+        self.w = torch.empty(nbytes // 4, dtype=torch.float32, device=device)
+        self.r = torch.zeros(nbytes // 4, dtype=torch.float32, device=device)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.amax()
 
 
 # ------------------------------------------------------------------ replicas
@@ -329,7 +348,7 @@ def workload_config(cfg, world: int) -> dict:
     return {"workload": "llama7b block prefill, bf16, d=4096, 32 heads x 128, f=11008, B=1, T=2048",
             "global_batch": cfg.B * world, "seq_len": cfg.T,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "l2": "flushed before every timed step (256 MB write)"}
+            "l2": "flushed before every timed step (256 MB write, then a 256 MB read)"}
 
 
 def bench_prefill_config(lb, cfg, args, peaks, dev, stream, flush, barrier, max_over_ranks,
@@ -362,7 +381,7 @@ def bench_prefill_config(lb, cfg, args, peaks, dev, stream, flush, barrier, max_
     l0 = blk.launch_count
     barrier()
     for i in range(args.steps):
-        flush.zero_()
+        flush()
         starts[i].record(stream)
         blk.prefill(x, y, kc, vc, lens)
         ends[i].record(stream)
@@ -374,7 +393,7 @@ def bench_prefill_config(lb, cfg, args, peaks, dev, stream, flush, barrier, max_
     blk.enable_timing(True)
     barrier()
     for i in range(args.steps):
-        flush.zero_()
+        flush()
         blk.prefill(x, y, kc, vc, lens)
         for name, t in blk.stage_times():
             stage_ms.setdefault(name, []).append(t)
@@ -477,7 +496,7 @@ def run_ours(args):
     kc = torch.zeros(cfg.B, cfg.n_kv_heads, cfg.T, cfg.head_dim, dtype=torch.bfloat16, device=dev)
     vc = torch.zeros_like(kc)
     lens = torch.zeros(cfg.B, dtype=torch.int32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(L2_FLUSH_BYTES, dev)
 
     def barrier():
         if world > 1:
@@ -504,7 +523,7 @@ def run_ours(args):
         launches0 = blk.launch_count
         barrier()
         for i in range(args.steps):
-            flush.zero_()  # evict L2 outside the timed interval
+            flush()  # evict L2 outside the timed interval
             starts[i].record(stream)
             blk.prefill(x, y, kc, vc, lens)
             ends[i].record(stream)
@@ -517,7 +536,7 @@ def run_ours(args):
         blk.enable_timing(True)
         barrier()
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             blk.prefill(x, y, kc, vc, lens)
             for name, ms in blk.stage_times():
                 stage_ms.setdefault(name, []).append(ms)
@@ -625,7 +644,7 @@ def run_ours(args):
     in_done = [torch.cuda.Event() for _ in range(2)]
     comp_done = [torch.cuda.Event() for _ in range(2)]
     out_done = [torch.cuda.Event() for _ in range(2)]
-    flush.zero_()
+    flush()
     torch.cuda.synchronize()
     barrier()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

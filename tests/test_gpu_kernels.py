@@ -62,6 +62,11 @@ ATTN_CASES = [
     (2, 2, 2, 130, 400, 512, 64),     # queries at an offset (chunked prefill)
     (3, 2, 1, 1, 513, 600, 128),      # a single decode-like query per sequence
     (1, 2, 2, 384, 384, 384, 128),    # exact tiles
+    (2, 2, 2, 130, 400, 512, 128),    # offset; consecutive-row CTA pairs, one key block
+                                      # after all rows of the first CTA
+    (1, 6, 2, 200, 333, 352, 128),    # offset, n_rep = 3 (odd: consecutive-row pairs)
+    (2, 4, 1, 129, 129, 160, 128),    # n_rep = 4 (head pairs), one row past a tile
+    (1, 4, 4, 600, 600, 640, 128),    # five 128-key blocks: every buffer and ring stage reused
 ]
 
 

@@ -56,12 +56,12 @@ CPU_SAMPLE_T = 2048  # tokens of the 7B prefill the CPU oracle evaluates per sam
 # the kernel's source file at capture time: once that file changes the figure no longer
 # describes the kernel and the bench reports null until it is captured again.
 NCU_TRAFFIC = {
-    # gemm_tc_pair_kernel<256, 2>, 7B prefill
-    "gate_up_swiglu_gemm": {"bytes": 198_123_776 + 35_764_480, "source": "gemm_tc.cu",
-                            "sha256": None},
-    # attn_decode_split_kernel<128, 1>, L=4096
-    "attention_decode": {"bytes": 2_148_352_000 + 8_126_464, "source": "attn_decode.cu",
-                         "sha256": None},
+    # gemm_tc_pair_kernel<256, 2>, 7B prefill (profiles/traffic_gate_up_llama7b_decode_attn_b32.md)
+    "gate_up_swiglu_gemm": {"bytes": 197_773_056 + 34_841_600, "source": "gemm_tc.cu",
+                            "sha256": "501a878ad9c656f9"},
+    # attn_decode_split_kernel<128, 1>, 7B decode B=32, L=4096 (same file)
+    "attention_decode": {"bytes": 2_148_306_176 + 7_738_624, "source": "attn_decode.cu",
+                         "sha256": "5ec1499e5ac75cd8"},
 }
 
 
@@ -411,6 +411,8 @@ def bench_prefill_config(lb, cfg, args, peaks, dev, stream, flush, barrier, max_
            "steps": args.steps, "kernel_launches": launches}
     if cfg.dtype == "bf16":
         out["frac_of_bf16_peak"] = tflops / peaks["bf16_tflops"]
+        if peaks.get("bf16_tflops_sustained"):  # the longer steps run under the power cap
+            out["frac_of_bf16_sustained_peak"] = tflops / peaks["bf16_tflops_sustained"]
         if "attention" in stages:
             at = flops["attn"] / (stages["attention"] * 1e-3) / 1e12
             out["attention"] = {"ms": stages["attention"], "gflop": flops["attn"] / 1e9, "tflops": at,
@@ -567,7 +569,7 @@ def run_ours(args):
                 blk.decode(xs[s], yd, kcd, vcd, dlens)
             blk.sync_status()
             reps = 2
-            dec_ms, attn_ms = [], []
+            dec_ms, attn_ms, dec_stage = [], [], {}
             dl0 = blk.launch_count
             barrier()
             for r in range(reps):
@@ -579,6 +581,7 @@ def run_ours(args):
                     blk.decode(xs[s], yd, kcd, vcd, dlens)
                     if r == reps - 1:
                         for name, ms in blk.stage_times():
+                            dec_stage.setdefault(name, []).append(ms)
                             if name == "attention":
                                 attn_ms.append(ms)
                 ev1.record(stream)
@@ -622,6 +625,7 @@ def run_ours(args):
                 "ms_per_step": per_step_ms, "hbm_gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
                 "bytes_per_step_mean": bytes_mean, "tokens_per_s": dcfg.B / (per_step_ms * 1e-3) * world,
                 "steps": args.decode_steps, "repetitions": reps, "kernel_launches": dec_launches,
+                "stage_ms": {k: round(statistics.mean(v), 4) for k, v in dec_stage.items()},
                 "attention_kernel": {"ms": statistics.mean(attn_ms), "bytes_mean": attn_bytes_mean,
                                      "achieved_gbs": attn_gbs, "frac": attn_gbs / peaks["hbm_gbs"],
                                      "traffic": ncu_traffic("attention_decode")},

@@ -520,7 +520,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();
+  if (warp != 0) pdl_wait();
 
   const int num_m = (M + 2 * kBM - 1) / (2 * kBM), num_n = (N + BN - 1) / BN;
   const int KB = (K + kBK - 1) / kBK;
@@ -529,20 +529,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer (both CTAs)
+      // The weight operand B is no output of the previous kernel: the B tiles of the
+      // first ring's worth of K blocks are requested before waiting for that kernel;
+      // their A tiles (the activations) follow once it has completed.
+      int npre = 0;
+      if (pair < units) {
+        const int nt0 = pair / num_m;
+        npre = min(KB, C::STAGES);
+        for (int kb = 0; kb < npre; ++kb) {  // fresh ring: every stage is free
+          if (rank == 0) mbar_arrive_expect_tx(&full[kb], 2 * C::STAGE_BYTES);
+          tma_load_2d_pair(sB + kb * C::B_BYTES, &tmB, pair_addr(&full[kb], 0), kb * kBK,
+                           nt0 * BN + rank * (BN / 2));
+        }
+      }
+      pdl_wait();
       uint32_t stage = 0, phase = 0;
       long long issued = 0;
       bool ok = true;
       for (int u = pair; u < units && ok; u += npairs) {
         const int mt = u % num_m, nt = u / num_m;
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, epi.err, 0x11)) {
-            ok = false;
-            break;
-          }
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
           const uint32_t fb = pair_addr(&full[stage], 0);
-          tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, fb, kb * kBK, mt * 2 * kBM + rank * kBM);
-          tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, fb, kb * kBK, nt * BN + rank * (BN / 2));
+          if (issued < npre) {  // B already requested
+            tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, fb, kb * kBK, mt * 2 * kBM + rank * kBM);
+          } else {
+            if (!mbar_wait(&empty[stage], phase ^ 1, epi.err, 0x11)) {
+              ok = false;
+              break;
+            }
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+            tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, fb, kb * kBK, mt * 2 * kBM + rank * kBM);
+            tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, fb, kb * kBK, nt * BN + rank * (BN / 2));
+          }
           ++issued;
           if (++stage == C::STAGES) {
             stage = 0;

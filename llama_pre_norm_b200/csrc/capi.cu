@@ -655,6 +655,7 @@ static lb_status run_prefill(llama_block* b, const void* x, void* y, int B, int 
     e1.q_out = w.q; e1.k_cache = k_cache; e1.v_cache = v_cache; e1.pos0 = L;
     e1.cos_t = b->cos_t; e1.sin_t = b->sin_t; e1.err = b->err;
     e1.row_ss = w.ss1; e1.row_inv_d = 1.f / d; e1.row_eps = b->eps;
+    e1.operands_ready = true;  // x and W_qkv: only the epilogue needs row_ssq's statistics
     LB_STAGE("qkv_rope_gemm", 1, launch_gemm_tc(x, b->w_qkv, M, b->n_qkv, d, 256, 1, e1, b->num_sms, s));
     LB_STAGE("attention", 1,
              launch_attn_tc(w.q, k_cache, v_cache, w.o, B, T, L + T, H, Hkv, dh, t_max, b->err, s));
@@ -872,6 +873,7 @@ lb_status llama_block_tp_attn_prefill(llama_block* b, const void* x, void* o_par
   e1.q_out = w.q; e1.k_cache = k_cache; e1.v_cache = v_cache; e1.pos0 = 0;
   e1.cos_t = b->cos_t; e1.sin_t = b->sin_t; e1.err = b->err;
   e1.row_ss = w.ss1; e1.row_inv_d = 1.f / d; e1.row_eps = b->eps;
+  e1.operands_ready = true;  // x and W_qkv: only the epilogue needs row_ssq's statistics
   LB_STAGE("qkv_rope_gemm", 1, launch_gemm_tc(x, b->w_qkv, M, b->n_qkv, d, 256, 1, e1, b->num_sms, s));
   LB_STAGE("attention", 1, launch_attn_tc(w.q, k_cache, v_cache, w.o, B, T, T, H, Hkv, dh, t_max, b->err, s));
   GemmEpi e2;  // this shard's o_proj columns: a partial sum, no residual

@@ -520,7 +520,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  if (warp != 0) pdl_wait();
+  if (warp >= 2 || (warp == 1 && !epi.operands_ready)) pdl_wait();
 
   const int num_m = (M + 2 * kBM - 1) / (2 * kBM), num_n = (N + BN - 1) / BN;
   const int KB = (K + kBK - 1) / kBK;
@@ -542,7 +542,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                            nt0 * BN + rank * (BN / 2));
         }
       }
-      pdl_wait();
+      if (!epi.operands_ready) pdl_wait();
       uint32_t stage = 0, phase = 0;
       long long issued = 0;
       bool ok = true;

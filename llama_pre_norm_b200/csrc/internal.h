@@ -160,6 +160,11 @@ struct GemmEpi {
   // kEpiResid: when ss_out != NULL, the sum of squares of each stored (rounded)
   // output row is accumulated into ss_out[m] (atomically, over the N tiles).
   float* ss_out = nullptr;
+  // Neither operand is written by the kernel launched just before this GEMM (which
+  // triggered its dependents only after its own wait, so everything earlier is complete):
+  // the TMA producer and the MMA issuer then start without waiting for that kernel; only
+  // the epilogue does (it reads row_ss).
+  bool operands_ready = false;
 };
 
 // D[M,N] = A[M,K] · B[N,K]^T, bf16 operands (K-major, row stride K), fp32 accumulation in

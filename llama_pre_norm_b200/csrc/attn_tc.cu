@@ -47,7 +47,7 @@
 
 namespace lb {
 
-constexpr int kAttnTcThreads = 352;
+constexpr int kAttnTcThreads = 480;
 constexpr float kRescaleLog2 = 8.0f;
 
 // ---------------------------------------------------------------- softmax arithmetic
@@ -89,8 +89,8 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_
       "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(hi), "r"(0u));
 }
 
-// Barrier for the 256 softmax threads (id 5).
-__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 5, 256;" ::: "memory"); }
+// Barrier for the 128 epilogue threads (id 5).
+__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 5, 128;" ::: "memory"); }
 
 template <int DH>
 struct AttnCfg {
@@ -101,7 +101,7 @@ struct AttnCfg {
   static constexpr int PANEL_BYTES = 128 * 128;  // one panel of a 128-row tile
   static constexpr int Q_BYTES = BQ * DH * 2;
   static constexpr int KV_BYTES = BKV * DH * 2;
-  static constexpr int XCH_FLOATS = 6 * 128;     // row-max swap [2 steps][2 halves], row sums [2]
+  static constexpr int XCH_FLOATS = 8 * 128;     // row maxima [2 steps][2 halves], row sums [2 units][2 halves]
   static constexpr int SMEM =
       2 * Q_BYTES + (KST + VST) * KV_BYTES + XCH_FLOATS * 4 + 256 + 1024;
   static constexpr int O_COL = NS * 128;         // S buffers at columns 0, 128, 256; O after
@@ -178,7 +178,9 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
   uint64_t* pv_ready = s_full + NS;
   uint64_t* o_full = pv_ready + NS;       // [NS]: PV(g) completes a phase of o_full[g % NS]
   uint64_t* o_free = o_full + NS;         // a unit's O has been read out of TMEM
-  uint64_t* drain = o_free + 1;
+  uint64_t* l_ready = o_free + 1;         // [2]: a unit's row sums handed to the epilogue
+  uint64_t* xsum_free = l_ready + 2;      // [2]: ... and read by it
+  uint64_t* drain = xsum_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -199,7 +201,11 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
       mbar_init(&pv_ready[i], 9);  // one arrival per softmax warp + the V load
       mbar_init(&o_full[i], 1);
     }
-    mbar_init(o_free, 8);
+    mbar_init(o_free, 4);  // one arrival per epilogue warp
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&l_ready[i], 8);    // softmax warps
+      mbar_init(&xsum_free[i], 4);  // epilogue warps
+    }
     mbar_init(drain, 1);
     fence_mbar_init();
     prefetch_tmap(&tmQ);
@@ -335,16 +341,15 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
       umma_commit(drain);
       mbar_wait(drain, 0, err, 0x28);
     }
-  } else {
-    // ---------------- softmax / correction / output: warps 2..5 keys 0..63, 6..9 keys 64..127
+  } else if (warp <= 9) {
+    // ---------------- softmax / correction: warps 2..5 keys 0..63, 6..9 keys 64..127
     const int hf = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // query row within the tile == TMEM lane
     const uint32_t lane_base = tmem_base + ((uint32_t)(quarter * 32) << 16);
     const uint32_t t_o = lane_base + C::O_COL + hf * (DH / 2);
     float* xmax = xch;            // [step % 2][half][row]
-    float* xsum = xch + 4 * 128;  // [half][row]
-    const bool storer = warp == 2 && lane == 0;  // issues the output tile's TMA stores
+    float* xsum = xch + 4 * 128;  // [unit % 2][half][row]
     bool ok = true;
     // PV(g) is waited on through o_full[g % NS]. A parity wait reads the right phase
     // only while its barrier is at most one phase ahead: the phase before (PV(g-NS))
@@ -407,21 +412,22 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
         // accumulators. P is packed in place as bf16 pairs (word k of chunk c: keys
         // 32c + 2k, 32c + 2k + 1) and stored over this half's first 32 score columns
         // (chunk c at column 16c, whose scores are already in registers).
-        const float nm = -m_new;
-        float rs0 = 0.f, rs1 = 0.f;
+        // The exponent arguments and the row sum use paired fp32 operations (one
+        // instruction per two keys).
+        const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_new, -m_new);
+        float2 rs = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float p0 = ex2_approx(fmaf(s[c][i], scale_log2, nm));
-            const float p1 = ex2_approx(fmaf(s[c][i + 1], scale_log2, nm));
-            rs0 += p0;
-            rs1 += p1;
-            s[c][i >> 1] = __uint_as_float(pack_bf16x2(p0, p1));
+            const float2 x = __ffma2_rn(make_float2(s[c][i], s[c][i + 1]), sc2, nm2);
+            const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            rs = __fadd2_rn(rs, p);
+            s[c][i >> 1] = __uint_as_float(pack_bf16x2(p.x, p.y));
           }
           tmem_st16(t_s + c * 16, *reinterpret_cast<const uint32_t(*)[16]>(s[c]));
         }
-        l_run = l_run * alpha + (rs0 + rs1);
+        l_run = l_run * alpha + (rs.x + rs.y);
         m_ref = m_new;
         if (j > 0 && __any_sync(0xffffffffu, move)) {
           // Rescale this half of O once it holds PV(g-1); PV(g) is only issued after
@@ -442,50 +448,70 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0 && ok) mbar_arrive(&pv_ready[buf]);
-        if (j == 0 && k > 0 && storer) {
-          // The previous unit's output tile has long been read out of its Q buffer:
-          // hand the buffer back to the producer for the Q after next.
-          bulk_wait_group_read0();
-          mbar_arrive(&q_empty[(k - 1) & 1]);
-        }
       }
-      // ---- unit end: O = sum over its steps of P V, normalised by the row sum
-      pv_wait(g - 1, 0x2b);
-      tc_fence_after();
-      float o[DH / 64][32];
-#pragma unroll
-      for (int c = 0; c < DH / 64; ++c) tmem_ld32(t_o + c * 32, o[c]);
-      tmem_wait_ld();
-      tc_fence_before();
+      // ---- unit end: hand the half row sum to the epilogue warps (slot k % 2, free
+      // once they have read unit k - 2's) and go on with the next unit at once
+      if (k >= 2 && ok) ok = mbar_wait_warp(&xsum_free[k & 1], ((k >> 1) & 1) ^ 1, err, 0x2e);
+      xsum[((k & 1) * 2 + hf) * 128 + r] = l_run;
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_free);  // the next unit's PVs may overwrite O now
-      xsum[hf * 128 + r] = l_run;
-      quarter_bar(quarter);
-      const float inv_l = 1.f / (l_run + xsum[(hf ^ 1) * 128 + r]);
-      // The normalised half row goes into the unit's Q buffer (its last QK^T has
-      // completed) in the 128-byte swizzled panel layout of the output tensor map,
-      // which the TMA store reads; rows past T_q are dropped by the store.
+      if (lane == 0) mbar_arrive(&l_ready[k & 1]);
+    }
+  } else {
+    // ---------------- epilogue: warps 11..14, one output row per thread. For each unit:
+    // wait for its last PV, read O out of TMEM (then O is free for the next unit's PVs),
+    // normalise by the row sum, write the row into the unit's Q buffer (its last QK^T
+    // has completed) in the 128-byte swizzled panel layout of the output tensor map,
+    // and store the tile with TMA; rows past T_q are dropped by the store. The Q buffer
+    // goes back to the producer once the store has read it.
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t t_o = tmem_base + ((uint32_t)(quarter * 32) << 16) + C::O_COL;
+    const float* xsum = xch + 4 * 128;
+    const bool storer = warp == 11 && lane == 0;
+    bool ok = true;
+    int g = 0;
+    for (int k = 0; k < nunits; ++k) {
+      const AttnUnit u = attn_unit(attn_unit_index(k, blockIdx.x, G), B, Tq, Tk, H, Hkv);
+      g += u.n;  // g - 1: the unit's last step
+      if (ok) ok = mbar_wait_warp(&l_ready[k & 1], (k >> 1) & 1, err, 0x2f);
+      const float inv_l = 1.f / (xsum[((k & 1) * 2) * 128 + r] + xsum[((k & 1) * 2 + 1) * 128 + r]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&xsum_free[k & 1]);
+      // PV(g-1) via o_full[(g-1) % NS]: the phase before (PV(g-4)) completed before the
+      // softmax could see S(g-1), and the phase after needs O released below.
+      if (ok) ok = mbar_wait_warp(&o_full[(g - 1) % NS], ((g - 1) / NS) & 1, err, 0x2b);
+      tc_fence_after();
       uint8_t* stage = sQ + (k & 1) * C::Q_BYTES;
-#pragma unroll
-      for (int c = 0; c < DH / 64; ++c) {
+#pragma unroll 1
+      for (int c = 0; c < DH / 32; ++c) {
+        float o[32];
+        tmem_ld32(t_o + c * 32, o);
+        tmem_wait_ld();
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int col = hf * (DH / 2) + c * 32 + q * 8;
+          const int col = c * 32 + q * 8;
           const int p = col >> 6, ch = (col & 63) >> 3;
           uint4 w;
-          w.x = pack_bf16x2(o[c][q * 8 + 0] * inv_l, o[c][q * 8 + 1] * inv_l);
-          w.y = pack_bf16x2(o[c][q * 8 + 2] * inv_l, o[c][q * 8 + 3] * inv_l);
-          w.z = pack_bf16x2(o[c][q * 8 + 4] * inv_l, o[c][q * 8 + 5] * inv_l);
-          w.w = pack_bf16x2(o[c][q * 8 + 6] * inv_l, o[c][q * 8 + 7] * inv_l);
+          w.x = pack_bf16x2(o[q * 8 + 0] * inv_l, o[q * 8 + 1] * inv_l);
+          w.y = pack_bf16x2(o[q * 8 + 2] * inv_l, o[q * 8 + 3] * inv_l);
+          w.z = pack_bf16x2(o[q * 8 + 4] * inv_l, o[q * 8 + 5] * inv_l);
+          w.w = pack_bf16x2(o[q * 8 + 6] * inv_l, o[q * 8 + 7] * inv_l);
           *reinterpret_cast<uint4*>(stage + p * C::PANEL_BYTES + r * 128 + ((ch ^ (r & 7)) * 16)) = w;
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);  // the next unit's PVs may overwrite O now
       fence_proxy_async_smem();  // generic-proxy writes, read next by the TMA engine
-      softmax_bar();
-      if (storer && ok) {
-        for (int p = 0; p < C::PANELS; ++p)
-          tma_store_3d(&tmO, stage + p * C::PANEL_BYTES, u.h * DH + p * 64, u.q0, u.b);
-        bulk_commit_group();
+      epilogue_bar();
+      if (storer) {
+        if (ok) {
+          for (int p = 0; p < C::PANELS; ++p)
+            tma_store_3d(&tmO, stage + p * C::PANEL_BYTES, u.h * DH + p * 64, u.q0, u.b);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+        mbar_arrive(&q_empty[k & 1]);  // for the Q after next
       }
     }
     if (storer) bulk_wait_group0();  // the last tile is written before the CTA exits

@@ -24,7 +24,9 @@ The other prefill shapes are timed the same way and reported beside the headline
 64 query / 8 KV heads, f=28672, B=1, T=4096) and ``prefill_tiny_f32`` (the fp32
 block, d=256, T=64), each with tokens/s, TFLOP/s, fraction of the bf16 peak, the
 per-stage times and, on a 1-GPU run, the fp64 oracle timed on 64 sampled rows per
-sequence with the GPU output's error at those rows.
+sequence with the GPU output's error at those rows. ``tp_prefill_shards`` (1-GPU runs)
+times rank 0's share of a tensor-parallel 7B and 70B prefill layer at 2, 4 and 8 ranks,
+with the layer's two all-reduces modelled at the measured peer bandwidth.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -349,6 +351,75 @@ def workload_config(cfg, world: int) -> dict:
             "global_batch": cfg.B * world, "seq_len": cfg.T,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": "flushed before every timed step (256 MB write, then a 256 MB read)"}
+
+
+NVLINK_GBS = 770.0  # measured peer copy per direction per GPU on this machine (900 nominal)
+
+
+def bench_tp_shard(lb, cfg, world: int, args, peaks, dev, stream, flush) -> dict:
+    """Per-rank compute of one tensor-parallel prefill layer at `world` ranks ("深入解析Llama
+    MLP模块" page §6.3 split): rank 0's shard (n_heads / W query heads, n_kv_heads / W KV
+    heads, f / W intermediate columns) runs llama_block_tp_attn_prefill and
+    llama_block_tp_mlp on one GPU, L2 flushed before each timed step, CUDA events on the
+    library's stream. The two all-reduces of the layer (the attention and MLP partial sums,
+    M x d bf16 each) are not run here (one GPU per run); their time is modelled as a ring
+    all-reduce at the measured peer-copy bandwidth and reported separately."""
+    import torch
+
+    H, Hkv, f = cfg.n_heads // world, cfg.n_kv_heads // world, cfg.f // world
+    sc = cfg.with_(name=f"{cfg.name} shard 0/{world}", n_heads=H, n_kv_heads=Hkv, f=f)
+    g = torch.Generator(device=dev).manual_seed(1234 + world)
+    def rnd(*shape):
+        return (torch.randn(*shape, generator=g, device=dev, dtype=torch.float32) * 0.02).to(torch.bfloat16)
+    d, dh = cfg.d, cfg.head_dim
+    Ws = {"wq": rnd(H * dh, d), "wk": rnd(Hkv * dh, d), "wv": rnd(Hkv * dh, d), "wo": rnd(d, H * dh),
+          "w_gate": rnd(f, d), "w_up": rnd(f, d), "w_down": rnd(d, f),
+          "g_attn": torch.ones(d, dtype=torch.bfloat16, device=dev),
+          "g_mlp": torch.ones(d, dtype=torch.bfloat16, device=dev)}
+    blk = lb.LlamaBlock(d, H, Hkv, dh, f, cfg.eps, cfg.rope_base, torch.bfloat16, max_pos=cfg.T)
+    blk.set_weights(Ws)
+    del Ws
+    x = (torch.randn(cfg.B, cfg.T, d, generator=g, device=dev)).to(torch.bfloat16)
+    o_part, x1, m_part = torch.empty_like(x), torch.empty_like(x), torch.empty_like(x)
+    kc = torch.zeros(cfg.B, Hkv, cfg.T, dh, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    lens = torch.zeros(cfg.B, dtype=torch.int32, device=dev)
+
+    def layer():
+        lens.zero_()
+        lb.llama_block_tp_attn_prefill(blk.handle, x, o_part, kc, vc, lens, stream=stream)
+        # o_part stands in for the all-reduced attention sum (same shape; values only scale X')
+        lb.llama_block_tp_mlp(blk.handle, x, o_part, x1, m_part, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            layer()
+    blk.sync_status()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    l0 = blk.launch_count
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush()
+            starts[i].record(stream)
+            layer()
+            ends[i].record(stream)
+    torch.cuda.synchronize()
+    launches = blk.launch_count - l0
+    blk.sync_status()
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    fl = prefill_flops(sc)["total"]
+    M = cfg.B * cfg.T
+    ar_bytes = 2 * M * d * 2  # two all-reduces of an M x d bf16 partial per layer
+    wire = ar_bytes * 2 * (world - 1) / world  # ring all-reduce: bytes each rank sends
+    ex_ms = wire / (NVLINK_GBS * 1e9) * 1e3
+    blk.close()
+    return {"world": world, "shard": f"{H} heads / {Hkv} KV heads x {dh}, f={f}",
+            "rank_compute_ms": ms, "tflops": fl / (ms * 1e-3) / 1e12,
+            "frac_of_bf16_peak": fl / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "allreduce_bytes_per_layer": ar_bytes,
+            "modelled_allreduce_ms": ex_ms,
+            "modelled_layer_ms_no_overlap": ms + ex_ms, "kernel_launches": launches}
 
 
 def bench_prefill_config(lb, cfg, args, peaks, dev, stream, flush, barrier, max_over_ranks,
@@ -689,6 +760,24 @@ def run_ours(args):
                 extra[key] = bench_prefill_config(lb, c, args, peaks, dev, stream, flush, barrier,
                                                   max_over_ranks, want_cpu)
                 torch.cuda.empty_cache()
+            # tensor-parallel shards: one rank's compute of a 7B / 70B prefill layer at W = 2, 4, 8
+            if world == 1:
+                tp = {"note": "rank 0's compute of one tensor-parallel prefill layer, timed on one GPU; "
+                              "the two all-reduces per layer are modelled (ring, 770 GB/s per direction), "
+                              "not run: every run here has one GPU"}
+                for key, c, one_ms in (("llama7b", cfg, tot_ms / args.steps),
+                                       ("llama70b", LLAMA70B, extra["prefill_70b"]["ms_per_step"])):
+                    rows = []
+                    for Wn in (2, 4, 8):
+                        r = bench_tp_shard(lb, c, Wn, args, peaks, dev, stream, flush)
+                        r["one_gpu_ms"] = one_ms
+                        r["modelled_speedup_vs_1_gpu"] = one_ms / r["modelled_layer_ms_no_overlap"]
+                        rows.append(r)
+                        torch.cuda.empty_cache()
+                    tp[key] = {"workload": f"{c.name}: B={c.B}, T={c.T}", "shards": rows}
+                tp["kernel_launches"] = sum(r["kernel_launches"] for k in ("llama7b", "llama70b")
+                                            for r in tp[k]["shards"])
+                extra["tp_prefill_shards"] = tp
     clk = clocks.summary()
 
     tokens = cfg.B * cfg.T

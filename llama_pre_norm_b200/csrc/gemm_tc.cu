@@ -28,6 +28,12 @@ namespace lb {
 
 constexpr int kBM = 128, kBK = 64;
 constexpr int kGemmThreads = 192;
+// The pair kernel drains each accumulator with two warps per TMEM lane quarter, each
+// taking half of the tile's columns: the epilogue of a pair's last tile is not hidden
+// behind another tile's MMAs, and with one warp per quarter it took about half as
+// long as the tile's MMAs (a residual epilogue at 256 columns, ~12 us).
+constexpr int kPairEpiWarps = 8;
+constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
 
 template <int BN>
 struct GemmCfg {
@@ -82,12 +88,13 @@ __device__ __forceinline__ void store_row32(bf16* row, int n, int ncols, const f
 
 template <int BN>
 __device__ __forceinline__ void epi_store_resid(uint32_t tb, int m, int nt, int M, int N,
-                                                const GemmEpi& e, bool with_resid) {
+                                                const GemmEpi& e, bool with_resid,
+                                                int c0 = 0, int c1 = BN / 32) {
   bf16* out = reinterpret_cast<bf16*>(e.out);
   const bf16* res = reinterpret_cast<const bf16*>(e.resid);
   float ssq = 0.f;
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = c0; c < c1; ++c) {
     float v[32];
     tmem_ld32(tb + c * 32, v);
     tmem_wait_ld();
@@ -122,39 +129,41 @@ __device__ __forceinline__ void epi_store_resid(uint32_t tb, int m, int nt, int 
 
 // Residual-add epilogue with the row's residual already in registers (rres: the
 // BN columns of row m, loaded before the accumulator was ready).
-template <int BN>
-__device__ __forceinline__ void prefetch_resid(uint4 (&rres)[BN / 8], int m, int nt, int M, int N,
-                                               const GemmEpi& e) {
+template <int BN, int NC>
+__device__ __forceinline__ void prefetch_resid(uint4 (&rres)[NC / 8], int m, int nt, int M, int N,
+                                               const GemmEpi& e, int c0) {
   const int n0 = nt * BN;
   if (m < M && n0 + BN <= N) {
     const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(e.resid) +
-                                                      (long long)m * e.ldo + n0);
+                                                      (long long)m * e.ldo + n0 + c0 * 32);
 #pragma unroll
-    for (int i = 0; i < BN / 8; ++i) rres[i] = src[i];
+    for (int i = 0; i < NC / 8; ++i) rres[i] = src[i];
   }
 }
 
-template <int BN>
+template <int BN, int NC>
 __device__ __forceinline__ void epi_resid_prefetched(uint32_t tb, int m, int nt, int M, int N,
-                                                     const GemmEpi& e, const uint4 (&rres)[BN / 8]) {
+                                                     const GemmEpi& e, const uint4 (&rres)[NC / 8],
+                                                     int c0) {
   const int n0 = nt * BN;
   // ragged tile (some row of this warp or the columns out of range): the general
   // path. The choice is warp-uniform: tcgen05.ld is a warp-collective instruction.
   if (!__all_sync(0xffffffffu, m < M && n0 + BN <= N)) {
-    epi_store_resid<BN>(tb, m, nt, M, N, e, true);
+    epi_store_resid<BN>(tb, m, nt, M, N, e, true, c0, c0 + NC / 32);
     return;
   }
   bf16* out = reinterpret_cast<bf16*>(e.out) + (long long)m * e.ldo;
   float ssq = 0.f;
-#pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+#pragma unroll  // static indices keep rres in registers
+  for (int cc = 0; cc < NC / 32; ++cc) {
+    const int c = c0 + cc;
     float v[32];
     tmem_ld32(tb + c * 32, v);
     tmem_wait_ld();
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       float r[8];
-      unpack_bf16x8(rres[c * 4 + q], r);
+      unpack_bf16x8(rres[cc * 4 + q], r);
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[q * 8 + i] += r[i];
     }
@@ -172,11 +181,11 @@ __device__ __forceinline__ void epi_resid_prefetched(uint32_t tb, int m, int nt,
 
 // Tile columns [0,128) are gate rows 128*nt.., [128,256) the matching up rows.
 __device__ __forceinline__ void epi_swiglu(uint32_t tb, int m, int nt, int M, int f,
-                                           const GemmEpi& e) {
+                                           const GemmEpi& e, int j0 = 0, int j1 = 4) {
   bf16* out = reinterpret_cast<bf16*>(e.out);
   const float r = row_scale(e, m, M);
 #pragma unroll 1
-  for (int j = 0; j < 4; ++j) {
+  for (int j = j0; j < j1; ++j) {
     float g[32], u[32];
     tmem_ld32(tb + j * 32, g);
     tmem_ld32(tb + 128 + j * 32, u);
@@ -195,16 +204,18 @@ __device__ __forceinline__ void epi_swiglu(uint32_t tb, int m, int nt, int M, in
 // i + dh/2 of the same head (rotate_half), both held by this thread.
 template <int BN>
 __device__ __forceinline__ void epi_qkv_rope(uint32_t tb, int m, int nt, int M, int N,
-                                             const GemmEpi& e) {
+                                             const GemmEpi& e, int part = 0, int nparts = 1) {
   const int dh = e.dh, half = dh >> 1;
   const int b = m / e.T, t = m - (m / e.T) * e.T;
   const int pos = e.pos0 + t;
   const bool row_ok = m < M;
   const float r = row_scale(e, m, M);
   bool pos_ok = pos < e.max_pos && pos < e.t_max;
-  if (row_ok && !pos_ok) latch_error(e.err, kErrCacheBounds);
+  if (row_ok && !pos_ok && part == 0) latch_error(e.err, kErrCacheBounds);
+  // heads of the tile taken by this part (BN / dh is 2 or 4, nparts 1 or 2)
+  const int nh = BN / dh, h0 = part * nh / nparts, h1 = (part + 1) * nh / nparts;
 #pragma unroll 1
-  for (int hh = 0; hh < BN / dh; ++hh) {
+  for (int hh = h0; hh < h1; ++hh) {
     const int gcol = nt * BN + hh * dh;
     if (gcol >= N) break;  // uniform across the warp
     const int hq = gcol / dh;
@@ -481,7 +492,7 @@ struct Gemm2Cfg {
 };
 
 template <int BN, int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, int M, int N, int K, GemmEpi epi) {
   using C = Gemm2Cfg<BN>;
@@ -508,7 +519,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA of the pair
+      mbar_init(&tempty[a], 2 * kPairEpiWarps);  // epilogue warps of both CTAs
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -613,35 +624,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_wait(drain, 0, epi.err, 0x15);
     }
   } else {
-    // ---------------- epilogue (warps 2..5 of both CTAs, 128 rows each)
-    const int quarter = warp & 3;
+    // ---------------- epilogue (warps 2.. of both CTAs, 128 rows each): warp w reads
+    // TMEM lane quarter w % 4 and takes part (w - 2) / 4 of the tile's columns
+    constexpr int kParts = kPairEpiWarps / 4;
+    const int quarter = warp & 3, part = (warp - 2) >> 2;
     const int row_in_tile = quarter * 32 + lane;
+    constexpr int NC = BN / kParts;  // columns per part
+    const int c0 = part * (NC / 32);
     int t = 0;
     for (int u = pair; u < units; u += npairs, ++t) {
       const int mt = u % num_m, nt = u / num_m;
       const int acc = t & 1;
       const int m = mt * 2 * kBM + rank * kBM + row_in_tile;
-      // With a short K loop (o_proj) the residual is fetched while the accumulator
-      // is still being computed; with a long one (down_proj) measurement showed the
-      // early loads cost more than they hide, so it is read in the epilogue.
-      const bool prefetch = EPI == kEpiResid && KB <= 64;
-      uint4 rres[EPI == kEpiResid ? BN / 8 : 1];
+      // The residual is fetched while the accumulator is still being computed.
+      const bool prefetch = EPI == kEpiResid;
+      uint4 rres[EPI == kEpiResid ? NC / 8 : 1];
       if constexpr (EPI == kEpiResid)
-        if (prefetch) prefetch_resid<BN>(rres, m, nt, M, N, epi);
+        if (prefetch) prefetch_resid<BN, NC>(rres, m, nt, M, N, epi, c0);
       if (!mbar_wait_warp(&tfull[acc], (t >> 1) & 1, epi.err, 0x16)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
       if constexpr (EPI == kEpiStore) {
-        epi_store_resid<BN>(tb, m, nt, M, N, epi, false);
+        epi_store_resid<BN>(tb, m, nt, M, N, epi, false, c0, c0 + NC / 32);
       } else if constexpr (EPI == kEpiResid) {
         if (prefetch)
-          epi_resid_prefetched<BN>(tb, m, nt, M, N, epi, rres);
+          epi_resid_prefetched<BN, NC>(tb, m, nt, M, N, epi, rres, c0);
         else
-          epi_store_resid<BN>(tb, m, nt, M, N, epi, true);
+          epi_store_resid<BN>(tb, m, nt, M, N, epi, true, c0, c0 + NC / 32);
       } else if constexpr (EPI == kEpiSwiGLU) {
-        epi_swiglu(tb, m, nt, M, epi.f, epi);
+        epi_swiglu(tb, m, nt, M, epi.f, epi, part * 4 / kParts, (part + 1) * 4 / kParts);
       } else {
-        epi_qkv_rope<BN>(tb, m, nt, M, N, epi);
+        epi_qkv_rope<BN>(tb, m, nt, M, N, epi, part, kParts);
       }
       tc_fence_before();
       __syncwarp();
@@ -678,7 +691,7 @@ static cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int M,
   static std::atomic<unsigned long long> attr_done{0};
   if (cudaError_t e = ensure_smem_attr(kern, C::SMEM, attr_done); e != cudaSuccess)
     return e;
-  return launch_k_pair(kern, grid, kGemmThreads, C::SMEM, s, ta, tb, M, N, K, epi);
+  return launch_k_pair(kern, grid, kPairThreads, C::SMEM, s, ta, tb, M, N, K, epi);
 }
 
 // 2-SM pair path: 256 x 256 tiles, no split-K.

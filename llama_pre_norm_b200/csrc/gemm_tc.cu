@@ -86,6 +86,45 @@ __device__ __forceinline__ void store_row32(bf16* row, int n, int ncols, const f
   }
 }
 
+// Coalesced output rows for the pair kernel's epilogue warps. A thread owns one output row,
+// so a direct 16-byte store of each thread touches 32 rows (32 cache lines) per
+// instruction, and those stores slowed the next tile's MMAs. Instead each warp puts two
+// 32-column pieces of its 32 rows (two 64-byte segments per row) as bf16 into its own
+// 4 KB of shared memory, 16-byte units XOR-swizzled by row (conflict-free on both sides),
+// then writes them out with 8 lanes per row: each instruction covers 4 rows x 128 bytes.
+constexpr int kStageBytes = 32 * 128;  // per epilogue warp
+
+__device__ __forceinline__ void stage_seg(uint8_t* sw, int lane, int seg, const float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+    const int unit = seg * 4 + q;
+    *reinterpret_cast<uint4*>(sw + lane * 128 + ((unit ^ (lane & 7)) << 4)) = u;
+  }
+}
+
+// Write the staged rows: segment 0 of row r to row_ptr(r)[0, 32), segment 1 to
+// row_ptr(r)[off1, off1 + 32), where row_ptr / ok are this lane's row (lane r owns row r).
+__device__ __forceinline__ void stage_flush(const uint8_t* sw, int lane, const bf16* row_ptr, int off1,
+                                            bool ok) {
+  __syncwarp();
+  const unsigned long long p = reinterpret_cast<unsigned long long>(row_ptr);
+  const int u = lane & 7;
+  const int col = (u >> 2) * off1 + (u & 3) * 8;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int r = it * 4 + (lane >> 3);
+    const uint4 val = *reinterpret_cast<const uint4*>(sw + r * 128 + ((u ^ (r & 7)) << 4));
+    bf16* base = reinterpret_cast<bf16*>(__shfl_sync(0xffffffffu, p, r));
+    const int okr = __shfl_sync(0xffffffffu, (int)ok, r);
+    if (okr) *reinterpret_cast<uint4*>(base + col) = val;
+  }
+  __syncwarp();  // the buffer may be refilled
+}
+
 template <int BN>
 __device__ __forceinline__ void epi_store_resid(uint32_t tb, int m, int nt, int M, int N,
                                                 const GemmEpi& e, bool with_resid,
@@ -144,7 +183,7 @@ __device__ __forceinline__ void prefetch_resid(uint4 (&rres)[NC / 8], int m, int
 template <int BN, int NC>
 __device__ __forceinline__ void epi_resid_prefetched(uint32_t tb, int m, int nt, int M, int N,
                                                      const GemmEpi& e, const uint4 (&rres)[NC / 8],
-                                                     int c0) {
+                                                     int c0, uint8_t* stage, int lane) {
   const int n0 = nt * BN;
   // ragged tile (some row of this warp or the columns out of range): the general
   // path. The choice is warp-uniform: tcgen05.ld is a warp-collective instruction.
@@ -174,16 +213,34 @@ __device__ __forceinline__ void epi_resid_prefetched(uint32_t tb, int m, int nt,
         ssq += v[i] * v[i];
       }
     }
-    store_row32(out, n0 + c * 32, N, v);
+    stage_seg(stage, lane, cc & 1, v);
+    if (cc & 1) stage_flush(stage, lane, out + n0 + (c - 1) * 32, 32, true);
   }
   if (e.ss_out && m < M) atomicAdd(e.ss_out + m, ssq);
 }
 
 // Tile columns [0,128) are gate rows 128*nt.., [128,256) the matching up rows.
 __device__ __forceinline__ void epi_swiglu(uint32_t tb, int m, int nt, int M, int f,
-                                           const GemmEpi& e, int j0 = 0, int j1 = 4) {
+                                           const GemmEpi& e, int j0 = 0, int j1 = 4,
+                                           uint8_t* stage = nullptr, int lane = 0) {
   bf16* out = reinterpret_cast<bf16*>(e.out);
   const float r = row_scale(e, m, M);
+  // staged, coalesced stores when the warp's columns are whole pairs of chunks in range
+  if (stage && ((j1 - j0) & 1) == 0 && nt * 128 + j1 * 32 <= f) {
+    bf16* row = out + (long long)m * e.ldo;
+#pragma unroll 1
+    for (int j = j0; j < j1; ++j) {
+      float g[32], u[32];
+      tmem_ld32(tb + j * 32, g);
+      tmem_ld32(tb + 128 + j * 32, u);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i] * r) * (u[i] * r);
+      stage_seg(stage, lane, (j - j0) & 1, g);
+      if ((j - j0) & 1) stage_flush(stage, lane, row + nt * 128 + (j - 1) * 32, 32, m < M);
+    }
+    return;
+  }
 #pragma unroll 1
   for (int j = j0; j < j1; ++j) {
     float g[32], u[32];
@@ -204,7 +261,8 @@ __device__ __forceinline__ void epi_swiglu(uint32_t tb, int m, int nt, int M, in
 // i + dh/2 of the same head (rotate_half), both held by this thread.
 template <int BN>
 __device__ __forceinline__ void epi_qkv_rope(uint32_t tb, int m, int nt, int M, int N,
-                                             const GemmEpi& e, int part = 0, int nparts = 1) {
+                                             const GemmEpi& e, int part = 0, int nparts = 1,
+                                             uint8_t* stage = nullptr, int lane = 0) {
   const int dh = e.dh, half = dh >> 1;
   const int b = m / e.T, t = m - (m / e.T) * e.T;
   const int pos = e.pos0 + t;
@@ -232,7 +290,45 @@ __device__ __forceinline__ void epi_qkv_rope(uint32_t tb, int m, int nt, int M, 
       rotate = false;
     }
     const bool store = row_ok && pos_ok;
-    if (rotate) {
+    if (stage) {  // staged, coalesced stores (every thread takes part; `store` masks rows)
+      if (rotate) {
+#pragma unroll 1
+        for (int j = 0; j < half / 32; ++j) {
+          float x1[32], x2[32];
+          tmem_ld32(tb + hh * dh + j * 32, x1);
+          tmem_ld32(tb + hh * dh + half + j * 32, x2);
+          tmem_wait_ld();
+          const float* ct = e.cos_t + (long long)(store ? pos : 0) * half + j * 32;
+          const float* st = e.sin_t + (long long)(store ? pos : 0) * half + j * 32;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float c[8], sn[8];
+            load8(ct + q * 8, c);
+            load8(st + q * 8, sn);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float a = x1[q * 8 + i] * r, bb = x2[q * 8 + i] * r;
+              x1[q * 8 + i] = a * c[i] - bb * sn[i];
+              x2[q * 8 + i] = bb * c[i] + a * sn[i];
+            }
+          }
+          stage_seg(stage, lane, 0, x1);
+          stage_seg(stage, lane, 1, x2);
+          stage_flush(stage, lane, dst + j * 32, half, store);
+        }
+      } else {
+#pragma unroll 1
+        for (int j = 0; j < dh / 32; ++j) {
+          float x[32];
+          tmem_ld32(tb + hh * dh + j * 32, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] *= r;
+          stage_seg(stage, lane, j & 1, x);
+          if (j & 1) stage_flush(stage, lane, dst + (j - 1) * 32, 32, store);
+        }
+      }
+    } else if (rotate) {
 #pragma unroll 1
       for (int j = 0; j < half / 32; ++j) {
         float x1[32], x2[32];
@@ -488,7 +584,9 @@ struct Gemm2Cfg {
   static constexpr int B_BYTES = (BN / 2) * kBK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 256 + 1024;
+  static constexpr int OUT_STAGE = kPairEpiWarps * kStageBytes;  // coalesced output rows
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 256 + OUT_STAGE + 1024;
+  static_assert(SMEM <= 232448, "pair GEMM exceeds the shared memory of a CTA");
 };
 
 template <int BN, int EPI>
@@ -631,6 +729,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int row_in_tile = quarter * 32 + lane;
     constexpr int NC = BN / kParts;  // columns per part
     const int c0 = part * (NC / 32);
+    uint8_t* stage = smem + C::STAGES * C::STAGE_BYTES + 256 + (warp - 2) * kStageBytes;
     int t = 0;
     for (int u = pair; u < units; u += npairs, ++t) {
       const int mt = u % num_m, nt = u / num_m;
@@ -648,13 +747,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         epi_store_resid<BN>(tb, m, nt, M, N, epi, false, c0, c0 + NC / 32);
       } else if constexpr (EPI == kEpiResid) {
         if (prefetch)
-          epi_resid_prefetched<BN, NC>(tb, m, nt, M, N, epi, rres, c0);
+          epi_resid_prefetched<BN, NC>(tb, m, nt, M, N, epi, rres, c0, stage, lane);
         else
           epi_store_resid<BN>(tb, m, nt, M, N, epi, true, c0, c0 + NC / 32);
       } else if constexpr (EPI == kEpiSwiGLU) {
-        epi_swiglu(tb, m, nt, M, epi.f, epi, part * 4 / kParts, (part + 1) * 4 / kParts);
+        epi_swiglu(tb, m, nt, M, epi.f, epi, part * 4 / kParts, (part + 1) * 4 / kParts, stage, lane);
       } else {
-        epi_qkv_rope<BN>(tb, m, nt, M, N, epi, part, kParts);
+        epi_qkv_rope<BN>(tb, m, nt, M, N, epi, part, kParts, stage, lane);
       }
       tc_fence_before();
       __syncwarp();

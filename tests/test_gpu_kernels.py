@@ -90,6 +90,30 @@ def test_causal_attn(dt, case):
     assert row_err(got, want.reshape(B, Tq, H, dh)) <= _tol(dt)
 
 
+@pytest.mark.parametrize("slope", [0.05, 1.0, 20.0])
+def test_causal_attn_scores_growing_along_keys(slope):
+    """Online-softmax reference moves: component 0 of key t is slope * t and of every
+    query +1 (even heads) or -1 (odd heads), so along the keys the scores grow (the
+    running max moves between 128-key steps: by about 0.6, 11 and 226 natural-log
+    units per step for the three slopes, the last far past the fp32 exponent range if
+    a step's exponentials were taken against the previous reference) or shrink (the
+    max stays at key 0). Compared with the fp64 oracle like every other attention case."""
+    dt = torch.bfloat16
+    B, H, Hkv, T, dh = 1, 4, 2, 600, 128
+    q = make_tensor((B, H, T, dh), 410, torch.float32, std=0.5)
+    k = make_tensor((B, Hkv, T, dh), 411, torch.float32, std=0.5)
+    v = make_tensor((B, Hkv, T, dh), 412, torch.float32)
+    q[:, 0::2, :, 0] = 1.0
+    q[:, 1::2, :, 0] = -1.0
+    k[:, :, :, 0] = slope * torch.arange(T, dtype=torch.float32)
+    q, k, v = q.to(dt), k.to(dt), v.to(dt)
+    o = torch.empty(B, T, H * dh, dtype=dt, device="cuda")
+    lb.causal_attn(cuda(q), cuda(k), cuda(v), o)
+    lb.llama_block_sync_status()
+    want = ob.causal_attention(q, k, v).transpose(0, 2, 1, 3).reshape(B, T, H, dh)
+    assert row_err(as_np(o).reshape(B, T, H, dh), want) <= BF16_TOL
+
+
 @pytest.mark.parametrize("dt,M,d,f", [
     (torch.float32, 17, 256, 688),
     (torch.bfloat16, 300, 512, 1000),   # ragged M, f not a multiple of 128

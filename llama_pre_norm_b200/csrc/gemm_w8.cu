@@ -228,8 +228,11 @@ __global__ void __launch_bounds__(kW8Threads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kt = kt0; kt < kt1; ++kt) {
-          if (!mbar_wait(&full[rs], rphase, epi.err, 0x44) ||
-              !mbar_wait(&a_full[rs], rphase, epi.err, 0x45)) {
+          // One wait: the converter group arrives on a_full only after it has waited for
+          // full (the INT8 tile and the token tile landed), so a completed a_full phase
+          // orders this step's token tile before the MMAs that read it. (The trace of a
+          // step: this thread issuing its MMAs is the step's slowest part.)
+          if (!mbar_wait(&a_full[rs], rphase, epi.err, 0x45)) {
             ok = false;
             break;
           }

@@ -16,6 +16,8 @@ llama_block_sync_status(NULL) reads and clears; and that calls whose partials
 would not fit, or whose K/V are misaligned, are refused on the host. This file
 is named so that pytest collects it last."""
 
+import gc
+
 import numpy as np
 import pytest
 import torch
@@ -57,6 +59,7 @@ def test_static_scratch_decode_attention_matches_oracle(B, H, Hkv, dh, L, ks):
         o.fill_(float("nan"))
         torch.cuda.synchronize()
         if call == 1:
+            gc.collect()  # tensors of earlier tests in reference cycles are freed now, not mid-call
             free_after_first = torch.cuda.mem_get_info()[0]
             alloc_after_first = torch.cuda.memory_allocated()
         lb.decode_attn_static_scratch(qd, kd, vd, o, kv_len)

@@ -12,9 +12,10 @@
 // r*G .. r*G + G - 1, forwards on even rounds and backwards on odd ones), and every
 // pipeline below runs across unit boundaries, so the next unit's Q load and first
 // score tiles overlap the current unit's last steps and its output write.
-//   warp 0       TMA producer: Q of the next unit into the second Q buffer, K one
-//                ring ahead of V (K_0, K_1, K_2, then V_g, K_{g+3} per step g). A K
-//                (V) stage is reused once the S (PV) product that read it completed.
+//   warp 0       TMA producer: the Q of units 0 and 1, then K one ring ahead of V (K_0,
+//                K_1, K_2, then V_g, K_{g+3} per step g). A K (V) stage is reused once
+//                the S (PV) product that read it completed. It never waits for a Q
+//                buffer: the epilogue loads the later units' Q (below).
 //   warp 10      issues S(g) = Q K^T into TMEM score buffer g % 3, so S(g+1) and
 //                S(g+2) are computed while the softmax works on S(g); S(g) overwrites
 //                P(g-3) and therefore waits for PV(g-3) to complete.
@@ -37,10 +38,14 @@
 //                TMEM, each half rescaling half of O's columns) when a row's max grows
 //                by more than 2^8, so most steps skip the rescale; P <= 2^8 stays exact
 //                enough in bf16 and the final O / l uses the same reference.
-//                At the end of a unit each thread reads its half row of O, releases O
-//                to the next unit's PVs, and writes the normalised row into the unit's
-//                Q buffer (no longer read by any MMA), from where one thread stores the
-//                tile with TMA while the softmax moves on to the next unit.
+//                At the end of a unit they hand their half-row sums to the epilogue
+//                warps (a two-slot ring in shared memory) and go on with the next unit.
+//   warps 11..14 epilogue: wait for the unit's last PV, read O out of TMEM (which
+//                releases it to the next unit's PVs), normalise, stage the rows in the
+//                unit's Q buffer (its last QK^T has completed) and store the tile with
+//                TMA. Once the store has read the buffer, the same thread loads the Q
+//                of unit k + 2 into it: a producer that waited for the buffer held
+//                back the K/V loads behind it and stalled the PVs at unit changes.
 #include "common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -168,8 +173,7 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
   float* xch = reinterpret_cast<float*>(sV + VST * C::KV_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(xch + C::XCH_FLOATS);
   uint64_t* q_full = bars;                // [2]
-  uint64_t* q_empty = q_full + 2;         // [2]: output tile stored out of the buffer
-  uint64_t* k_full = q_empty + 2;         // [KST]
+  uint64_t* k_full = q_full + 2;          // [KST]
   // A K stage is free once the S product that read it has completed (s_full), a V
   // stage once its PV product has (o_full): the producer waits on those barriers.
   uint64_t* s_full = k_full + KST;        // [NS] score buffers
@@ -191,10 +195,7 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
   const int nunits = rounds + (((rounds & 1) ? G - 1 - (int)blockIdx.x : (int)blockIdx.x) < rem);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1);
-    }
+    for (int i = 0; i < 2; ++i) mbar_init(&q_full[i], 1);
     for (int i = 0; i < KST; ++i) mbar_init(&k_full[i], 1);
     for (int i = 0; i < NS; ++i) {
       mbar_init(&s_full[i], 1);
@@ -223,9 +224,10 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
   if (warp == 0) {
     if (lane == 0 && nunits > 0) {
       // ---------------- TMA producer
+      // Q of units 0 and 1 (both buffers are free); the epilogue's storer loads the Q of
+      // unit k + 2 into unit k's buffer once the output staged there has been stored.
       auto load_q = [&](int k, const AttnUnit& u) -> bool {
         const int qb = k & 1;
-        if (!mbar_wait(&q_empty[qb], ((k >> 1) & 1) ^ 1, err, 0x21)) return false;
         mbar_arrive_expect_tx(&q_full[qb], C::Q_BYTES);
         for (int p = 0; p < C::PANELS; ++p)
           tma_load_3d(sQ + qb * C::Q_BYTES + p * C::PANEL_BYTES, &tmQ, &q_full[qb], p * 64, u.q0,
@@ -252,18 +254,14 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
       vc.init(nunits, B, Tq, Tk, H, Hkv);
       kc.init(nunits, B, Tq, Tk, H, Hkv);
       bool ok = load_q(0, vc.u);
+      if (nunits > 1) load_q(1, attn_unit(attn_unit_index(1, blockIdx.x, G), B, Tq, Tk, H, Hkv));
       for (int i = 0; i < NS && ok && kc.valid(); ++i, kc.advance()) ok = load_kv(true, kc);
       int last_g = -1;  // last step whose V was issued
       for (; ok && vc.valid(); vc.advance()) {
         ok = load_kv(false, vc);
         if (!ok) break;
         last_g = vc.g;
-        if (vc.j == 0 && vc.k + 1 < nunits) {
-          // the next unit's Q, once its buffer's previous output has been stored
-          ok = load_q(vc.k + 1, attn_unit(attn_unit_index(vc.k + 1, blockIdx.x, G), B, Tq, Tk,
-                                           H, Hkv));
-        }
-        if (ok && kc.valid()) {
+        if (kc.valid()) {
           ok = load_kv(true, kc);
           kc.advance();
         }
@@ -510,8 +508,14 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
             tma_store_3d(&tmO, stage + p * C::PANEL_BYTES, u.h * DH + p * 64, u.q0, u.b);
           bulk_commit_group();
           bulk_wait_group_read0();
+          if (k + 2 < nunits) {  // the buffer is free: the Q of unit k + 2
+            const AttnUnit u2 = attn_unit(attn_unit_index(k + 2, blockIdx.x, G), B, Tq, Tk, H, Hkv);
+            mbar_arrive_expect_tx(&q_full[k & 1], C::Q_BYTES);
+            for (int p = 0; p < C::PANELS; ++p)
+              tma_load_3d(stage + p * C::PANEL_BYTES, &tmQ, &q_full[k & 1], p * 64, u2.q0,
+                          u2.b * H + u2.h);
+          }
         }
-        mbar_arrive(&q_empty[k & 1]);  // for the Q after next
       }
     }
     if (storer) bulk_wait_group0();  // the last tile is written before the CTA exits

@@ -58,7 +58,7 @@ CPU_SAMPLE_T = 2048  # tokens of the 7B prefill the CPU oracle evaluates per sam
 # the kernel's source file at capture time: once that file changes the figure no longer
 # describes the kernel and the bench reports null until it is captured again.
 NCU_TRAFFIC = {
-    # gemm_tc_pair_kernel<256, 2>, 7B prefill (profiles/traffic_gate_up_llama7b_decode_attn_b32.md)
+    # gemm_tc_pair_kernel<256, 2>, 7B prefill (a --set full capture of the current source)
     "gate_up_swiglu_gemm": {"bytes": 197_526_784 + 37_168_128, "source": "gemm_tc.cu",
                             "sha256": "b704e33952a75bd4"},
     # attn_decode_split_kernel<128, 1>, 7B decode B=32, L=4096 (same file)

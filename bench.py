@@ -61,7 +61,7 @@ NCU_TRAFFIC = {
     # gemm_tc_pair_kernel<256, 2>, 7B prefill (a --set full capture of the current source)
     "gate_up_swiglu_gemm": {"bytes": 197_526_784 + 37_168_128, "source": "gemm_tc.cu",
                             "sha256": "b704e33952a75bd4"},
-    # attn_decode_split_kernel<128, 1>, 7B decode B=32, L=4096 (same file)
+    # attn_decode_split_kernel<128, 1>, 7B decode B=32, L=4096 (a --metrics capture)
     "attention_decode": {"bytes": 2_148_306_176 + 7_738_624, "source": "attn_decode.cu",
                          "sha256": "5ec1499e5ac75cd8"},
 }
